@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse FP8-KV MLA decode hot path on B200.
+
+One step = the whole hot path over one batch of synthetic input:
+scheduler metadata -> split-KV decode kernel -> PDL-chained combine, through
+the library's public API (the C ABI via the Python binding).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the float64 CPU oracle, timed on host cores
+
+Rank 0 prints one JSON line.  With N > 1 (launched by torch.distributed.run)
+every rank runs its own independent replica of the workload (different
+seeds, no data-path collective): requests are independent, so the path shards
+with no exchange and the scaling is weak.  `value` is the FLOP of all ranks'
+steps divided by the slowest rank's time.
+
+Timing: W warm-up steps, then exactly K steps bracketed by a barrier and a
+device synchronisation, timed with CUDA events on the launching stream.  The
+inputs rotate over several independent copies (each with its own cache,
+queries and indices) whose combined size exceeds the 126 MB L2, so a step's
+gathered rows were not left in L2 by the previous steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import signal
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse FP8-KV MLA decode TFLOP/s (% of BF16 TC peak) and gathered-KV GB/s"
+DQK, DV, ROW = 576, 512, 656
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode_h128_b64_topk2048")
+    ap.add_argument("--copies", type=int, default=4, help="independent input copies rotated over the steps")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def valid_counts(idx: np.ndarray, seqlens: np.ndarray) -> np.ndarray:
+    sl = np.asarray(seqlens, dtype=np.int64).reshape(-1, 1, 1)
+    return ((idx >= 0) & (idx < sl)).sum(axis=-1)
+
+
+def step_flops(h_q: int, valid: np.ndarray) -> float:
+    """Algorithmic FLOP of one step: 2 * h_q * valid_topk * (576 + 512) summed over query tokens."""
+    return float(2.0 * h_q * (DQK + DV) * valid.astype(np.float64).sum())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(hbm_gbs=float(pk["hbm_gbs"]), bf16_tflops=float(pk["bf16_tflops"]),
+                    bf16_tflops_sustained=float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.send_signal(signal.SIGTERM)
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.remove(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        sm = [r[0] for r in rows]
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the float64 CPU oracle
+# ---------------------------------------------------------------------------
+
+def host_inputs(w):
+    """Host copies of a workload for the oracle (cache rows from the oracle's own quantiser)."""
+    import oracle
+    from sparse_mla_decoding_b200 import workloads as W
+    lay = W.layout(w)
+    rows = lay.num_blocks * W.BLOCK
+    cache = np.empty((rows, ROW), dtype=np.uint8)
+    for start, lat, rope in W.cache_values(w, rows, chunk_rows=W.GEN_CHUNK_ROWS * 4):
+        cache[start:start + lat.shape[0]] = oracle.quantize_tokens_bulk(lat, rope)
+    W.poison(cache, W.unused_rows(lay))
+    idx = W.indices(w, lay.seqlens)
+    return dict(q=W.queries(w), cache=cache.reshape(lay.num_blocks, W.BLOCK, ROW), bt=lay.block_table,
+                seqlens=lay.seqlens.astype(np.int32), idx=idx)
+
+
+def cpu_oracle_sample(w, hi, budget_s: float, max_tokens=None):
+    """Time the oracle (single-threaded, as it stands) on tokens until the budget is spent."""
+    import oracle
+    tokens = [(b, t) for b in range(w.batch) for t in range(w.s_q)]
+    rng = np.random.default_rng(2024)
+    order = rng.permutation(len(tokens))
+    done, flops = 0, 0.0
+    t0 = time.perf_counter()
+    for k in order:
+        b, t = tokens[k]
+        oracle.sparse_decode_token(hi["q"][b, t], hi["cache"], hi["bt"][b], int(hi["seqlens"][b]), hi["idx"][b, t])
+        v = int(((hi["idx"][b, t] >= 0) & (hi["idx"][b, t] < hi["seqlens"][b])).sum())
+        flops += 2.0 * w.h_q * (DQK + DV) * v
+        done += 1
+        if time.perf_counter() - t0 >= budget_s or (max_tokens and done >= max_tokens):
+            break
+    dt = time.perf_counter() - t0
+    return flops, dt, done
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    hi = host_inputs(w)
+    n_tok = w.batch * w.s_q
+    per_step_budget = max(0.2, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, hi, per_step_budget / 4, max_tokens=1)
+    tot_f, tot_t, tot_n = 0.0, 0.0, 0
+    for _ in range(args.steps):
+        f, t, n = cpu_oracle_sample(w, hi, per_step_budget)
+        tot_f, tot_t, tot_n = tot_f + f, tot_t + t, tot_n + n
+    tflops = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q, "topk": w.topk},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{tot_n} of {n_tok} query tokens per pass over {args.steps} steps "
+                                   f"(single-threaded float64 C oracle)"},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def make_device_copy(w, device):
+    """Generator values -> device tensors; the cache rows are written by the library's own KV writer."""
+    import torch
+    import sparse_mla_decoding_b200 as smla
+    from sparse_mla_decoding_b200 import workloads as W
+    lay = W.layout(w)
+    rows = lay.num_blocks * W.BLOCK
+    cache = torch.empty((lay.num_blocks, W.BLOCK, ROW), dtype=torch.uint8, device=device)
+    flat = cache.view(rows, ROW)
+    for start, lat, rope in W.cache_values(w, rows, chunk_rows=W.GEN_CHUNK_ROWS * 4):
+        n = lat.shape[0]
+        dl = torch.from_numpy(lat.view(np.int16)).to(device).view(torch.bfloat16)
+        dr = torch.from_numpy(rope.view(np.int16)).to(device).view(torch.bfloat16)
+        smla.quantize_kv(dl, dr, flat[start:start + n])
+    unused = torch.from_numpy(W.unused_rows(lay)).to(device)
+    flat[unused] = torch.from_numpy(W.POISON_ROW).to(device)
+    idx = W.indices(w, lay.seqlens)
+    q = torch.from_numpy(W.queries(w).view(np.int16)).to(device).view(torch.bfloat16)
+    return dict(q=q, kvcache=cache, block_table=torch.from_numpy(lay.block_table).to(device),
+                cache_seqlens=torch.from_numpy(lay.seqlens.astype(np.int32)).to(device),
+                indices=torch.from_numpy(idx).to(device), idx_host=idx, seqlens_host=lay.seqlens)
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import sparse_mla_decoding_b200 as smla
+    from sparse_mla_decoding_b200 import workloads as W
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    smla.lib()
+    stream = torch.cuda.current_stream(device)
+
+    # independent copies (weak scaling: every rank has its own seeds)
+    copies = []
+    for c in range(args.copies):
+        wc = w.with_(seed=w.seed + 1000 * rank + 17 * c)
+        copies.append(make_device_copy(wc, device))
+    torch.cuda.synchronize()
+    flops_per_copy = [step_flops(w.h_q, valid_counts(c["idx_host"], c["seqlens_host"])) for c in copies]
+    valid_per_copy = [float(valid_counts(c["idx_host"], c["seqlens_host"]).sum()) for c in copies]
+    topk = w.topk
+    num_parts = smla.default_num_sm_parts(w.h_q, device)
+    ws = smla.new_workspace(w.batch, w.s_q, w.h_q, topk, num_parts, device)
+    outs = (torch.empty((w.batch, w.s_q, w.h_q, DV), dtype=torch.bfloat16, device=device),
+            torch.empty((w.batch, w.s_q, w.h_q), dtype=torch.float32, device=device))
+
+    def step(c):
+        d = copies[c]
+        sm, ns = smla.get_mla_metadata(d["cache_seqlens"], topk, w.h_q, num_parts, s_q=w.s_q)
+        return smla.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"],
+                                           d["indices"], sm, ns, workspace=ws, out=outs)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        step(i % args.copies)
+    torch.cuda.synchronize()
+
+    # ---- the timed region --------------------------------------------------
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i % args.copies)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    clocks = clk.summary()
+    my_flops = sum(flops_per_copy[i % args.copies] for i in range(args.steps))
+    my_valid = sum(valid_per_copy[i % args.copies] for i in range(args.steps))
+
+    # ---- the decode call alone (split kernel + chained combine), for the roofline
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    metas = [smla.get_mla_metadata(copies[c]["cache_seqlens"], topk, w.h_q, num_parts, s_q=w.s_q)
+             for c in range(args.copies)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        d, (sm, ns) = copies[i % args.copies], metas[i % args.copies]
+        evs[i][0].record(stream)
+        smla.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"], sm, ns,
+                                    workspace=ws, out=outs)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    kern_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+    # ---- end to end: pinned host inputs in, results out, every step --------
+    e2e = None
+    host = []
+    for c in copies:
+        host.append(dict(q=c["q"].cpu().pin_memory(), indices=c["indices"].cpu().pin_memory(),
+                         block_table=c["block_table"].cpu().pin_memory(),
+                         cache_seqlens=c["cache_seqlens"].cpu().pin_memory()))
+    dq = torch.empty_like(copies[0]["q"])
+    di = torch.empty_like(copies[0]["indices"])
+    dbt = [torch.empty_like(c["block_table"]) for c in copies]
+    dsl = torch.empty_like(copies[0]["cache_seqlens"])
+    ho = torch.empty(outs[0].shape, dtype=outs[0].dtype).pin_memory()
+    hl = torch.empty(outs[1].shape, dtype=outs[1].dtype).pin_memory()
+    h2d = (host[0]["q"].numel() * 2 + host[0]["indices"].numel() * 4 + host[0]["block_table"].numel() * 4 +
+           host[0]["cache_seqlens"].numel() * 4)
+    d2h = ho.numel() * 2 + hl.numel() * 4
+
+    def e2e_step(c):
+        h = host[c]
+        dq.copy_(h["q"], non_blocking=True)
+        di.copy_(h["indices"], non_blocking=True)
+        dbt[c].copy_(h["block_table"], non_blocking=True)
+        dsl.copy_(h["cache_seqlens"], non_blocking=True)
+        sm, ns = smla.get_mla_metadata(dsl, topk, w.h_q, num_parts, s_q=w.s_q)
+        o, l = smla.flash_mla_with_kvcache(dq, copies[c]["kvcache"], dbt[c], dsl, di, sm, ns, workspace=ws, out=outs)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(l, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i % args.copies)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i % args.copies)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    status, raw = smla.get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status word set during the benchmark: {raw:#x}")
+
+    # ---- reduce over ranks (max time, summed work) --------------------------
+    vals = torch.tensor([ms_total, e2e_ms, kern_ms, my_flops, my_valid], dtype=torch.float64, device=device)
+    if world > 1:
+        mx = vals.clone()
+        dist.all_reduce(mx[:3], op=dist.ReduceOp.MAX)
+        sm_ = vals.clone()
+        dist.all_reduce(sm_[3:], op=dist.ReduceOp.SUM)
+        vals = torch.cat([mx[:3], sm_[3:]])
+    ms_total, e2e_ms, kern_ms, tot_flops, tot_valid = vals.tolist()
+    if rank != 0:
+        return
+
+    peaks = load_peaks()
+    tflops = tot_flops / (ms_total * 1e-3) / 1e12
+    gbs = tot_valid * ROW / (ms_total * 1e-3) / 1e9
+    # roofline of the decode call on this rank: per-launch algorithmic work / average launch duration
+    per_launch_flops = float(np.mean(flops_per_copy))
+    per_launch_bytes = float(np.mean(valid_per_copy)) * ROW
+    intensity = (2.0 * w.h_q * (DQK + DV)) / ROW
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if intensity >= ridge:
+        achieved = per_launch_flops / (kern_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"]}
+    else:
+        achieved = per_launch_bytes / (kern_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    roof.update({"traffic": None, "kernel": "splitkv_mla_kernel + combine_kernel (one decode call)",
+                 "kernel_ms": kern_ms, "peak_source": peaks["source"] + " (burst)"})
+
+    line = {
+        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q, "topk": w.topk,
+                   "seqlen": int(copies[0]["seqlens_host"].max()), "kv_row_bytes": ROW, "num_sm_parts": num_parts,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs rotated over {args.copies} independent copies "
+                         f"({args.copies} x {copies[0]['kvcache'].numel() / 1e6:.0f} MB cache) > 126 MB L2"},
+        "gathered_kv_gbs": gbs,
+        "pct_of_bf16_peak": 100.0 * tflops / world / peaks["bf16_tflops"],
+        "roofline": roof,
+        "e2e": {"value": tot_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        hi = host_inputs(w.with_(seed=w.seed))
+        f, t, n = cpu_oracle_sample(w, hi, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{n} of {w.batch * w.s_q} query tokens of the same workload, "
+                                          f"{t:.1f} s single-threaded float64 C oracle"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    from sparse_mla_decoding_b200 import workloads as W
+    w = W.BY_NAME[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

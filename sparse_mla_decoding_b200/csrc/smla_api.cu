@@ -1,0 +1,245 @@
+// smla_api.cu -- the C ABI of libsmla.so (declared in include/smla.h): host-side
+// argument checks, workspace layout and kernel launches.  No device memory is
+// allocated and no stream is synchronised here (except where a function's
+// contract says so).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/smla.h"
+#include "sm100.cuh"
+#include "splitkv_mla.h"
+
+namespace smla {
+__global__ void sched_meta_kernel(int R, int n, int P, int32_t* sched_meta, int32_t* num_splits);
+__global__ void combine_kernel(const int32_t* num_splits, const float* o_accum, const float* lse_accum, int h_q,
+                               int max_splits, __nv_bfloat16* o, float* lse);
+__global__ void quantize_kv_kernel(const __nv_bfloat16* latent, const __nv_bfloat16* rope, int64_t n_tokens,
+                                   const int64_t* slot_mapping, uint8_t* kvcache, int64_t num_rows);
+__global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns);
+}  // namespace smla
+
+namespace {
+
+constexpr size_t kHeaderBytes = 256;
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_smem_configured[kMaxDevices];
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool valid_h_q(int h_q) { return h_q == 16 || h_q == 32 || h_q == 64 || h_q == 128; }
+
+int head_groups(int h_q) { return (h_q + 63) / 64; }
+
+int64_t n_tiles_of(int topk) { return ((int64_t)topk + SMLA_INDEX_TILE - 1) / SMLA_INDEX_TILE; }
+
+struct WorkspaceLayout {
+  size_t o_accum_off, lse_accum_off, total;
+};
+
+WorkspaceLayout workspace_layout(int batch, int s_q, int h_q, int num_sm_parts) {
+  const size_t max_splits = (size_t)batch * s_q + (size_t)num_sm_parts;
+  WorkspaceLayout w;
+  w.o_accum_off = kHeaderBytes;
+  const size_t o_bytes = max_splits * (size_t)h_q * SMLA_D_V * sizeof(float);
+  w.lse_accum_off = w.o_accum_off + ((o_bytes + 255) & ~size_t(255));
+  const size_t l_bytes = max_splits * (size_t)h_q * sizeof(float);
+  w.total = w.lse_accum_off + ((l_bytes + 255) & ~size_t(255));
+  return w;
+}
+
+int ensure_kernel_attributes() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SMLA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SMLA_ERR_UNSUPPORTED;
+  if (g_smem_configured[dev].load(std::memory_order_acquire)) return SMLA_OK;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) return SMLA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(smla::splitkv_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smla::splitkv_smem_bytes()) != cudaSuccess)
+    return SMLA_ERR_CUDA;
+  g_smem_configured[dev].store(1, std::memory_order_release);
+  return SMLA_OK;
+}
+
+cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute a;
+  std::memset(&a, 0, sizeof(a));
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* smla_status_string(int status) {
+  switch (status) {
+    case SMLA_OK: return "SMLA_OK";
+    case SMLA_ERR_INVALID_ARGUMENT: return "SMLA_ERR_INVALID_ARGUMENT";
+    case SMLA_ERR_UNSUPPORTED: return "SMLA_ERR_UNSUPPORTED";
+    case SMLA_ERR_CUDA: return "SMLA_ERR_CUDA";
+    case SMLA_ERR_DEVICE_TIMEOUT: return "SMLA_ERR_DEVICE_TIMEOUT";
+    default: return "SMLA_UNKNOWN_STATUS";
+  }
+}
+
+int smla_version(void) { return 100; }
+
+int smla_default_num_sm_parts(int h_q, int device) {
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0) return -1;
+  const int per_part = head_groups(h_q > 0 ? h_q : 64);
+  const int parts = sms / per_part;
+  return parts > 0 ? parts : 1;
+}
+
+size_t smla_workspace_bytes(int batch, int s_q, int h_q, int topk, int num_sm_parts) {
+  if (batch < 0 || s_q < 1 || !valid_h_q(h_q) || topk < 1 || num_sm_parts < 1) return 0;
+  return workspace_layout(batch, s_q, h_q, num_sm_parts).total;
+}
+
+int smla_get_mla_metadata(const int32_t* cache_seqlens, int batch, int s_q, int topk, int h_q, int num_sm_parts,
+                          int32_t* sched_meta, int32_t* num_splits, void* stream) {
+  (void)cache_seqlens;
+  if (batch < 0 || s_q < 1 || topk < 1 || num_sm_parts < 1 || !sched_meta || !num_splits)
+    return SMLA_ERR_INVALID_ARGUMENT;
+  if (!valid_h_q(h_q)) return SMLA_ERR_UNSUPPORTED;
+  if (!aligned(sched_meta, 16)) return SMLA_ERR_INVALID_ARGUMENT;
+  const int64_t R = (int64_t)batch * s_q;
+  if (R > (1 << 28) || R * n_tiles_of(topk) > ((int64_t)1 << 40)) return SMLA_ERR_INVALID_ARGUMENT;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(256);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  if (cudaLaunchKernelEx(&cfg, smla::sched_meta_kernel, (int)R, (int)n_tiles_of(topk), num_sm_parts, sched_meta,
+                         num_splits) != cudaSuccess)
+    return SMLA_ERR_CUDA;
+  return SMLA_OK;
+}
+
+int smla_flash_mla_with_kvcache(const void* q, const uint8_t* kvcache, int64_t num_blocks, const int32_t* block_table,
+                                int max_blocks, const int32_t* cache_seqlens, const int32_t* indices,
+                                const int32_t* sched_meta, const int32_t* num_splits, int num_sm_parts,
+                                float softmax_scale, int batch, int s_q, int h_q, int topk, void* o, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_h_q(h_q)) return SMLA_ERR_UNSUPPORTED;
+  if (batch < 0 || s_q < 1 || topk < 1 || num_sm_parts < 1 || max_blocks < 1 || num_blocks < 1)
+    return SMLA_ERR_INVALID_ARGUMENT;
+  if (batch == 0) return SMLA_OK;
+  if (!q || !kvcache || !block_table || !cache_seqlens || !indices || !sched_meta || !num_splits || !o || !lse ||
+      !workspace)
+    return SMLA_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(kvcache, 16) || !aligned(o, 16) || !aligned(sched_meta, 16) ||
+      !aligned(workspace, 256))
+    return SMLA_ERR_INVALID_ARGUMENT;
+  const WorkspaceLayout wl = workspace_layout(batch, s_q, h_q, num_sm_parts);
+  if (workspace_bytes < wl.total) return SMLA_ERR_INVALID_ARGUMENT;
+  const int64_t R = (int64_t)batch * s_q;
+  if (R > (1 << 28) || n_tiles_of(topk) > (1 << 24)) return SMLA_ERR_INVALID_ARGUMENT;
+  if (int rc = ensure_kernel_attributes()) return rc;
+
+  float scale = softmax_scale;
+  if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)SMLA_D_QK);
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  smla::SplitKVParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kv = kvcache;
+  p.num_blocks = num_blocks;
+  p.block_table = block_table;
+  p.max_blocks = max_blocks;
+  p.seqlens = cache_seqlens;
+  p.indices = indices;
+  p.sched_meta = sched_meta;
+  p.num_splits = num_splits;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.topk = topk;
+  p.n_tiles = (int)n_tiles_of(topk);
+  p.num_parts = num_sm_parts;
+  p.num_requests = (int)R;
+  p.max_splits = (int)(R + num_sm_parts);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.o_accum = reinterpret_cast<float*>(ws + wl.o_accum_off);
+  p.lse_accum = reinterpret_cast<float*>(ws + wl.lse_accum_off);
+  p.status = reinterpret_cast<uint32_t*>(ws);
+
+  cudaLaunchAttribute attr = pdl_attribute();
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(num_sm_parts, head_groups(h_q));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smla::splitkv_smem_bytes();
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, smla::splitkv_mla_kernel, p) != cudaSuccess) return SMLA_ERR_CUDA;
+
+  cudaLaunchConfig_t ccfg;
+  std::memset(&ccfg, 0, sizeof(ccfg));
+  ccfg.gridDim = dim3((unsigned)R, h_q);
+  ccfg.blockDim = dim3(128);
+  ccfg.stream = static_cast<cudaStream_t>(stream);
+  ccfg.attrs = &attr;
+  ccfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&ccfg, smla::combine_kernel, (const int32_t*)num_splits, (const float*)p.o_accum,
+                         (const float*)p.lse_accum, h_q, p.max_splits, p.o, lse) != cudaSuccess)
+    return SMLA_ERR_CUDA;
+  return SMLA_OK;
+}
+
+int smla_quantize_kv(const void* latent, const void* rope, int64_t n_tokens, const int64_t* slot_mapping,
+                     uint8_t* kvcache, int64_t num_rows, void* stream) {
+  if (n_tokens < 0 || num_rows < 0) return SMLA_ERR_INVALID_ARGUMENT;
+  if (n_tokens == 0) return SMLA_OK;
+  if (!latent || !rope || !kvcache) return SMLA_ERR_INVALID_ARGUMENT;
+  if (!aligned(latent, 16) || !aligned(rope, 16) || !aligned(kvcache, 16)) return SMLA_ERR_INVALID_ARGUMENT;
+  if (!slot_mapping && n_tokens > num_rows) return SMLA_ERR_INVALID_ARGUMENT;
+  const int64_t blocks = (n_tokens + 7) / 8;
+  if (blocks > 0x7FFFFFFF) return SMLA_ERR_INVALID_ARGUMENT;
+  smla::quantize_kv_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(latent), static_cast<const __nv_bfloat16*>(rope), n_tokens, slot_mapping,
+      kvcache, num_rows);
+  return cudaGetLastError() == cudaSuccess ? SMLA_OK : SMLA_ERR_CUDA;
+}
+
+int smla_get_device_status(const void* workspace, int* status_out, uint32_t* raw_flags_out, void* stream) {
+  if (!workspace || !status_out) return SMLA_ERR_INVALID_ARGUMENT;
+  uint32_t flags = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return SMLA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SMLA_ERR_CUDA;
+  if (raw_flags_out) *raw_flags_out = flags;
+  if (flags & smla::kStatusTimeout) *status_out = SMLA_ERR_DEVICE_TIMEOUT;
+  else if (flags & (smla::kStatusBadBlockTable | smla::kStatusBadSchedule)) *status_out = SMLA_ERR_INVALID_ARGUMENT;
+  else *status_out = SMLA_OK;
+  return SMLA_OK;
+}
+
+int smla_reset_device_status(void* workspace, void* stream) {
+  if (!workspace) return SMLA_ERR_INVALID_ARGUMENT;
+  if (cudaMemsetAsync(workspace, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SMLA_ERR_CUDA;
+  return SMLA_OK;
+}
+
+int smla_selftest_bounded_wait(void* workspace, uint64_t limit_ns, void* stream) {
+  if (!workspace || limit_ns < 1 || limit_ns > 10000000000ull) return SMLA_ERR_INVALID_ARGUMENT;
+  smla::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t*>(workspace),
+                                                                              limit_ns);
+  return cudaGetLastError() == cudaSuccess ? SMLA_OK : SMLA_ERR_CUDA;
+}
+
+}  // extern "C"

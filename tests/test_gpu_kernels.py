@@ -1,0 +1,207 @@
+"""GPU parity of every kernel against the float64 oracle, through the C-ABI binding.
+
+  * scheduler metadata: bit-exact against the oracle's restatement
+  * KV writer (quantiser): bit-exact against the oracle's scalar quantiser
+  * bounded device wait: gives up, flags the status word, GPU stays usable
+  * split-KV decode + combine: o / lse within the stated tolerances on small
+    workloads spanning several tiles and a ragged tail, every head count,
+    split and unsplit schedules, invalid slots, all-invalid tokens, poisoned
+    unused rows, exact single-slot outputs and run-to-run bitwise determinism
+"""
+import numpy as np
+import pytest
+
+import oracle
+from sparse_mla_decoding_b200 import workloads as W
+
+import parity_util as PU
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    import torch
+    assert torch.cuda.is_available()
+    return torch
+
+
+@pytest.fixture(scope="module")
+def smla(torch_cuda):
+    import sparse_mla_decoding_b200 as m
+    m.lib()
+    return m
+
+
+# ---------------------------------------------------------------------------
+# scheduler
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("batch,s_q,topk,P", [(2, 1, 64, 148), (64, 1, 2048, 74), (128, 2, 2048, 148),
+                                              (32, 1, 2048, 74), (1, 4096, 2048, 74), (7, 3, 100, 5),
+                                              (1, 1, 1, 1), (5, 1, 7 * 64, 35), (13, 1, 128, 3),
+                                              (3, 1, 6400, 7), (200, 1, 64, 16), (9, 1, 1000, 300)])
+def test_sched_meta_bit_exact(smla, torch_cuda, batch, s_q, topk, P):
+    torch = torch_cuda
+    seqlens = torch.full((batch,), 100, dtype=torch.int32, device="cuda")
+    sm, ns = smla.get_mla_metadata(seqlens, topk, 64, P, s_q=s_q)
+    sm_ref, ns_ref = oracle.sched_meta(batch * s_q, -(-topk // 64), P)
+    assert np.array_equal(sm.cpu().numpy(), sm_ref)
+    assert np.array_equal(ns.cpu().numpy(), ns_ref)
+
+
+# ---------------------------------------------------------------------------
+# KV writer
+# ---------------------------------------------------------------------------
+
+def test_quantize_kv_bit_exact(smla, torch_cuda):
+    torch = torch_cuda
+    rng = np.random.default_rng(7)
+    n = 777
+    lat = rng.standard_normal((n, 512)).astype(np.float32) * np.float32(2.0)
+    lat[::5, 3] *= 8.0
+    lat[1, :128] = 0.0
+    lat[2, :] = 0.0
+    lat[3, 128:256] = 2.0 ** -120
+    lat[4, 256:384] = -0.0
+    lat[5, 384:] = np.float32(3e38)
+    lat[6, 7] = -448.0
+    lat_bits = W._to_bf16_bits(lat)
+    rope_bits = W._to_bf16_bits(rng.standard_normal((n, 64)).astype(np.float32))
+    ref = oracle.quantize_tokens(lat_bits, rope_bits)
+    dev_lat = torch.from_numpy(lat_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    dev_rope = torch.from_numpy(rope_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    cache = torch.zeros((n, 656), dtype=torch.uint8, device="cuda")
+    smla.quantize_kv(dev_lat, dev_rope, cache)
+    got = cache.cpu().numpy()
+    assert np.array_equal(got, ref)
+    # scattered writes through a slot mapping; negative slots are skipped
+    perm = rng.permutation(n + 40)[:n].astype(np.int64)
+    perm[::9] = -1
+    cache2 = torch.full((n + 40, 656), 0xAB, dtype=torch.uint8, device="cuda")
+    smla.quantize_kv(dev_lat, dev_rope, cache2, torch.from_numpy(perm).cuda())
+    got2 = cache2.cpu().numpy()
+    for i in range(n):
+        if perm[i] >= 0:
+            assert np.array_equal(got2[perm[i]], ref[i])
+    untouched = np.setdiff1d(np.arange(n + 40), perm[perm >= 0])
+    assert (got2[untouched] == 0xAB).all()
+
+
+# ---------------------------------------------------------------------------
+# bounded wait
+# ---------------------------------------------------------------------------
+
+def test_bounded_wait_gives_up_and_flags(smla, torch_cuda):
+    torch = torch_cuda
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    assert smla.get_device_status(ws) == (0, 0)
+    smla.selftest_bounded_wait(ws, 2_000_000)       # 2 ms
+    torch.cuda.synchronize()
+    st, raw = smla.get_device_status(ws)
+    assert st == 4 and raw & 1
+    smla.reset_device_status(ws)
+    assert smla.get_device_status(ws) == (0, 0)
+    # the context is still usable
+    assert float(torch.ones(4, device="cuda").sum()) == 4.0
+
+
+# ---------------------------------------------------------------------------
+# decode parity
+# ---------------------------------------------------------------------------
+
+def _check(w, num_sm_parts=None, tokens=None, indices=None, softmax_scale=None):
+    hi = PU.build_host_inputs(w, indices=indices)
+    o, lse, sm, ns = PU.run_gpu(hi, num_sm_parts=num_sm_parts, softmax_scale=softmax_scale)
+    toks = tokens or [(b, t) for b in range(w.batch) for t in range(w.s_q)]
+    ref = PU.oracle_tokens(hi, toks, softmax_scale=softmax_scale)
+    return hi, o, lse, PU.compare(o, lse, ref, w.name), ns
+
+
+def test_tiny_workload_all_tokens(smla):
+    _check(W.TINY)
+
+
+@pytest.mark.parametrize("h_q", [16, 32, 64, 128])
+@pytest.mark.parametrize("topk", [1, 64, 100, 300])
+def test_heads_and_ragged_topk(smla, h_q, topk):
+    w = W.Workload(f"ragged_h{h_q}_k{topk}", batch=3, s_q=2, h_q=h_q, topk=topk, seed=100 + topk,
+                   seqlens=(700, 130, 1000), index_mode="uniform", invalid_per_token=topk // 10)
+    _check(w)
+
+
+@pytest.mark.parametrize("P", [1, 2, 5, 37, 148])
+def test_split_schedules(smla, P):
+    w = W.Workload("splits", batch=4, s_q=1, h_q=64, topk=640, seed=77, seqlens=(2000, 1500, 700, 3000),
+                   index_mode="uniform", invalid_per_token=40)
+    _, _, _, _, ns = _check(w, num_sm_parts=P)
+    if P >= 37:
+        assert (np.diff(ns) > 1).any(), "expected at least one split request"
+
+
+def test_h128_long_topk_many_splits(smla):
+    w = W.Workload("h128_2048", batch=3, s_q=1, h_q=128, topk=2048, seed=91, seqlens=(8192, 4100, 2500),
+                   index_mode="uniform", outlier_channels=5)
+    _check(w)
+
+
+def test_invalid_slots_and_all_invalid_tokens(smla):
+    w = W.Workload("invalid", batch=3, s_q=2, h_q=64, topk=192, seed=5, seqlens=(300, 64, 1000),
+                   index_mode="uniform")
+    lay = W.layout(w)
+    idx = W.indices(w, lay.seqlens)
+    idx[0, 0, :] = -1                                  # every slot skipped -> o = 0, lse = -inf
+    idx[1, 1, :] = np.arange(64, 64 + 192)             # all at or past seqlen 64 -> invalid
+    idx[2, 0, ::3] = -5                                # other negative values are skips too
+    idx[2, 1, 10:20] = 10 ** 6                         # far past the length
+    _check(w, indices=idx)
+
+
+def test_single_valid_slot_is_exact(smla):
+    w = W.Workload("single", batch=2, s_q=1, h_q=32, topk=96, seed=8, seqlens=(500, 90), index_mode="uniform")
+    lay = W.layout(w)
+    idx = np.full((2, 1, 96), -1, np.int32)
+    idx[0, 0, 70] = 321
+    idx[1, 0, 0] = 89
+    hi = PU.build_host_inputs(w, indices=idx)
+    o, lse, _, _ = PU.run_gpu(hi)
+    for b, pos in ((0, 321), (1, 89)):
+        phys = hi.block_table[b, pos // 64] * 64 + pos % 64
+        v = oracle.dequantize_row(hi.cache.reshape(-1, 656)[phys])[:512]
+        assert np.array_equal(o[b, 0], np.broadcast_to(v, o[b, 0].shape))   # P = 1 exactly, V exact in bf16
+
+
+def test_softmax_scale_argument(smla):
+    w = W.TINY.with_(name="tiny_scale")
+    _check(w, softmax_scale=0.11)
+
+
+def test_bad_block_table_entry_is_skipped_and_flagged(smla, torch_cuda):
+    torch = torch_cuda
+    w = W.Workload("badbt", batch=1, s_q=1, h_q=16, topk=64, seed=9, seqlens=(256,), index_mode="uniform")
+    hi = PU.build_host_inputs(w)
+    bt = hi.block_table.copy()
+    bt[0, 2] = 10 ** 6                                  # past the cache
+    d = PU.to_device(hi)
+    d["block_table"] = torch.from_numpy(bt).cuda()
+    import sparse_mla_decoding_b200 as m
+    sm, ns = m.get_mla_metadata(d["cache_seqlens"], 64, 16, s_q=1)
+    ws = m.new_workspace(1, 1, 16, 64, sm.shape[0])
+    o, lse = m.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"],
+                                      sm, ns, workspace=ws)
+    st, raw = m.get_device_status(ws)
+    assert st == 1 and raw & 2
+    # the skipped slots are those whose block is the bad one: oracle with them marked invalid
+    idx = hi.indices.copy()
+    idx[(idx >= 128) & (idx < 192)] = -1
+    ref = PU.oracle_tokens(PU.HostInputs(hi.w, hi.q_bits, hi.cache, hi.block_table, hi.seqlens, idx), [(0, 0)])
+    PU.compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref, "badbt")
+
+
+def test_bitwise_deterministic(smla, torch_cuda):
+    w = W.Workload("det", batch=4, s_q=1, h_q=128, topk=1024, seed=12, seqlens=(4096,) * 4, index_mode="uniform")
+    hi = PU.build_host_inputs(w)
+    d = PU.to_device(hi)
+    o1, l1, _, _ = PU.run_gpu(hi, dev_inputs=d)
+    o2, l2, _, _ = PU.run_gpu(hi, dev_inputs=d)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
