@@ -55,7 +55,8 @@ typedef enum {
   SMLA_ERR_INVALID_ARGUMENT = 1, /* a null pointer, a bad size or an inconsistent shape */
   SMLA_ERR_UNSUPPORTED = 2,      /* h_q not in {16, 32, 64, 128}, or a device that is not sm_100 */
   SMLA_ERR_CUDA = 3,             /* a CUDA runtime call or a kernel launch failed */
-  SMLA_ERR_DEVICE_TIMEOUT = 4    /* reported by smla_get_device_status: a bounded device wait gave up */
+  SMLA_ERR_DEVICE_TIMEOUT = 4,   /* reported by smla_get_device_status: a bounded device wait gave up */
+  SMLA_ERR_SCRATCH_LIMIT = 5     /* the call needs more than SMLA_STATIC_SCRATCH_BYTES of library scratch */
 } smla_status;
 
 /* Head dimensions fixed by the operation. */
@@ -65,6 +66,8 @@ typedef enum {
 #define SMLA_KV_ROW_BYTES 656   /* 512 e4m3 | 4 x float32 scale | 64 x bf16 RoPE */
 #define SMLA_BLOCK_SIZE 64      /* tokens per paged-cache block */
 #define SMLA_INDEX_TILE 64      /* index slots per scheduling tile */
+/* Size of the library-owned device scratch of smla_flash_mla_with_kvcache_static_scratch. */
+#define SMLA_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* smla_status_string(int status);
@@ -165,6 +168,37 @@ int smla_quantize_kv(const void* latent, const void* rope, int64_t n_tokens, con
  *   workspace : device, as passed to smla_flash_mla_with_kvcache
  */
 int smla_get_device_status(const void* workspace, int* status_out, uint32_t* raw_flags_out, void* stream);
+
+/*
+ * Allocation-free variant of smla_flash_mla_with_kvcache.  The pages
+ * describe no counterpart; it exists for callers that cannot allocate device
+ * memory -- allocator-less runtimes and embedders that hand the library only
+ * their inputs and outputs, code where an allocation would synchronise or is
+ * not allowed, hosts whose memory planner owns every device byte.  Instead of
+ * a caller workspace it uses a fixed array of SMLA_STATIC_SCRATCH_BYTES
+ * (64 MiB) in the library's own device memory, which every GPU that loads
+ * the library holds until the process exits.  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *   Arguments as for smla_flash_mla_with_kvcache, without the workspace, plus
+ *   status_out : device uint32 (may be NULL).  If given, the kernels OR their
+ *                status flags (see smla_get_device_status) into it; the
+ *                caller zeroes it.  If NULL, the flags go to the scratch
+ *                header, which each call clears first and nothing reads back.
+ * The scratch need is the same as smla_workspace_bytes(batch, s_q, h_q, topk,
+ * num_sm_parts); a call that needs more returns SMLA_ERR_SCRATCH_LIMIT and
+ * launches nothing.  Every call on a device shares the one array and it keeps
+ * the last call's contents: calls whose kernels overlap on the GPU (other
+ * streams, other host threads) race on it and must be serialised by the
+ * caller.  The first call on each device does a one-time set-up with that
+ * device current (it looks up the array's device address and sets a kernel
+ * attribute), so make that first call before any stream capture.
+ */
+int smla_flash_mla_with_kvcache_static_scratch(const void* q, const uint8_t* kvcache, int64_t num_blocks,
+                                               const int32_t* block_table, int max_blocks,
+                                               const int32_t* cache_seqlens, const int32_t* indices,
+                                               const int32_t* sched_meta, const int32_t* num_splits,
+                                               int num_sm_parts, float softmax_scale, int batch, int s_q, int h_q,
+                                               int topk, void* o, float* lse, uint32_t* status_out, void* stream);
 
 /* Clear the workspace status word (asynchronously, on `stream`). */
 int smla_reset_device_status(void* workspace, void* stream);

@@ -87,6 +87,7 @@ const char* smla_status_string(int status) {
     case SMLA_ERR_UNSUPPORTED: return "SMLA_ERR_UNSUPPORTED";
     case SMLA_ERR_CUDA: return "SMLA_ERR_CUDA";
     case SMLA_ERR_DEVICE_TIMEOUT: return "SMLA_ERR_DEVICE_TIMEOUT";
+    case SMLA_ERR_SCRATCH_LIMIT: return "SMLA_ERR_SCRATCH_LIMIT";
     default: return "SMLA_UNKNOWN_STATUS";
   }
 }
