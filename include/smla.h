@@ -123,7 +123,8 @@ int smla_get_mla_metadata(const int32_t* cache_seqlens, int batch, int s_q, int 
  * were split.  Output is bitwise reproducible run to run (static schedule,
  * no floating-point atomics).
  *   q             : device bf16 [batch][s_q][h_q][576]
- *   kvcache       : device uint8 [num_blocks][64][656] (16-byte aligned)
+ *   kvcache       : device uint8 [num_blocks][64][656] (16-byte aligned);
+ *                   num_blocks <= 33554431 (rows are numbered with 32 bits)
  *   block_table   : device int32 [batch][max_blocks]
  *   cache_seqlens : device int32 [batch]
  *   indices       : device int32 [batch][s_q][topk]; -1 (any negative) or a

@@ -61,9 +61,7 @@ int ensure_kernel_attributes() {
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
   if (major != 10 || minor != 0) return SMLA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(smla::splitkv_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smla::splitkv_smem_bytes()) != cudaSuccess)
-    return SMLA_ERR_CUDA;
+  if (smla::configure_splitkv() != cudaSuccess) return SMLA_ERR_CUDA;
   g_smem_configured[dev].store(1, std::memory_order_release);
   return SMLA_OK;
 }
@@ -133,7 +131,9 @@ int smla_flash_mla_with_kvcache(const void* q, const uint8_t* kvcache, int64_t n
                                 float softmax_scale, int batch, int s_q, int h_q, int topk, void* o, float* lse,
                                 void* workspace, size_t workspace_bytes, void* stream) {
   if (!valid_h_q(h_q)) return SMLA_ERR_UNSUPPORTED;
-  if (batch < 0 || s_q < 1 || topk < 1 || num_sm_parts < 1 || max_blocks < 1 || num_blocks < 1)
+  // cache rows are addressed as 32-bit row numbers (block * 64 + offset)
+  if (batch < 0 || s_q < 1 || topk < 1 || num_sm_parts < 1 || max_blocks < 1 || num_blocks < 1 ||
+      num_blocks > (int64_t)(0x7FFFFFFF / SMLA_BLOCK_SIZE))
     return SMLA_ERR_INVALID_ARGUMENT;
   if (batch == 0) return SMLA_OK;
   if (!q || !kvcache || !block_table || !cache_seqlens || !indices || !sched_meta || !num_splits || !o || !lse ||
@@ -176,16 +176,8 @@ int smla_flash_mla_with_kvcache(const void* q, const uint8_t* kvcache, int64_t n
   p.lse_accum = reinterpret_cast<float*>(ws + wl.lse_accum_off);
   p.status = reinterpret_cast<uint32_t*>(ws);
 
+  if (smla::launch_splitkv(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SMLA_ERR_CUDA;
   cudaLaunchAttribute attr = pdl_attribute();
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(num_sm_parts, head_groups(h_q));
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = smla::splitkv_smem_bytes();
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, smla::splitkv_mla_kernel, p) != cudaSuccess) return SMLA_ERR_CUDA;
 
   cudaLaunchConfig_t ccfg;
   std::memset(&ccfg, 0, sizeof(ccfg));

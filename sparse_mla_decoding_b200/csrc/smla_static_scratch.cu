@@ -54,9 +54,7 @@ int setup_device(int dev, void** scratch_out) {
     g_scratch_addr[dev] = ptr;
   }
   if (!g_smem_set[dev]) {
-    if (cudaFuncSetAttribute(smla::splitkv_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smla::splitkv_smem_bytes()) != cudaSuccess)
-      return SMLA_ERR_CUDA;
+    if (smla::configure_splitkv() != cudaSuccess) return SMLA_ERR_CUDA;
     g_smem_set[dev] = true;
   }
   *scratch_out = g_scratch_addr[dev];
@@ -71,7 +69,9 @@ extern "C" int smla_flash_mla_with_kvcache_static_scratch(
     int num_sm_parts, float softmax_scale, int batch, int s_q, int h_q, int topk, void* o, float* lse,
     uint32_t* status_out, void* stream) {
   if (!(h_q == 16 || h_q == 32 || h_q == 64 || h_q == 128)) return SMLA_ERR_UNSUPPORTED;
-  if (batch < 0 || s_q < 1 || topk < 1 || num_sm_parts < 1 || max_blocks < 1 || num_blocks < 1)
+  // cache rows are addressed as 32-bit row numbers (block * 64 + offset)
+  if (batch < 0 || s_q < 1 || topk < 1 || num_sm_parts < 1 || max_blocks < 1 || num_blocks < 1 ||
+      num_blocks > (int64_t)(0x7FFFFFFF / SMLA_BLOCK_SIZE))
     return SMLA_ERR_INVALID_ARGUMENT;
   if (batch == 0) return SMLA_OK;
   if (!q || !kvcache || !block_table || !cache_seqlens || !indices || !sched_meta || !num_splits || !o || !lse)
@@ -143,15 +143,7 @@ extern "C" int smla_flash_mla_with_kvcache_static_scratch(
   std::memset(&attr, 0, sizeof(attr));
   attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr.val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(num_sm_parts, (h_q + 63) / 64);
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = smla::splitkv_smem_bytes();
-  cfg.stream = s;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, smla::splitkv_mla_kernel, p) != cudaSuccess) return SMLA_ERR_CUDA;
+  if (smla::launch_splitkv(p, s) != cudaSuccess) return SMLA_ERR_CUDA;
   cudaLaunchConfig_t ccfg;
   std::memset(&ccfg, 0, sizeof(ccfg));
   ccfg.gridDim = dim3((unsigned)R, h_q);

@@ -8,34 +8,49 @@
 //     数据加载 -- the 656-byte row: 512 e4m3 values dequantised to bf16 with
 //             their 1x128 tile scales, concatenated with the 64 bf16 RoPE
 //             values into the 576-wide key; bf16 MMAs with fp32 accumulation;
+//             loads carry an evict-first L2 hint;
+//     计算环节一 (Crossover) -- the 128 query heads of a token read the same
+//             K/V, so two CTAs of a cluster each own 64 heads, each
+//             dequantises half of the rows and writes them into both CTAs'
+//             shared memory;
 //     计算环节二 (Seesaw) -- the result is the FlashAttention online softmax;
 //     合并与性能账本 -- each split leaves a partial output and its lse.
 //   "deepseek-ai/FlashMLA" (agentlenshq), 技術的な詳細 -- -1 in indices marks
 //     an entry the kernel ignores.
 //
-// Design on B200 (not the Hopper design of the pages):
-//   * One CTA owns up to 64 query heads of one request at a time (M = 64 of
-//     every tcgen05.mma); 128 heads use two CTAs per scheduler part.
-//   * Per tile of 64 index slots: the slots are mapped through the block
-//     table, the 656-byte rows are gathered with 16-byte coalesced loads (one
-//     warp per row, one lane per 16 latent bytes), dequantised exactly
-//     (e4m3 -> f16 -> f32, times the tile scale in f32, round to bf16) and
-//     stored as a 64 x 576 bf16 K tile in the 128-byte-swizzled K-major
-//     layout the tensor core reads.  The same tile, read MN-major, is V.
-//   * S = Q K^T (M=64, N=64, K=576) and O += P V (M=64, N=256 twice, K=64)
-//     run as tcgen05.mma with fp32 accumulators in tensor memory.  The
-//     64 x 512 output accumulator takes 256 TMEM columns: its two 256-wide
-//     halves sit in the same columns, in the lower and upper 16 lanes of each
-//     32-lane sub-partition (the M=64 accumulator uses 16 lanes per
-//     sub-partition), which leaves room for S.
-//   * Online softmax in base 2 by the four warps that own the TMEM lanes;
-//     P is rounded to bf16 once and the same rounded values feed both the PV
-//     MMA and the running denominator.
+// Design on B200:
+//   * A CTA owns 64 query heads of one request at a time (M = 64 of every
+//     tcgen05.mma).  128 heads run as a two-CTA cluster (one CTA per 64-head
+//     group) that shares the dequantised tiles over distributed shared memory;
+//     16/32 heads are zero-padded to 64 in a single CTA.
+//   * Warp roles (288 threads):
+//       warps 0-3  softmax: online softmax over S in TMEM, P to shared memory,
+//                  lazy O rescaling, epilogue (own TMEM lane quarters 0-3);
+//       warps 4-7  producers: index -> page map, 16-byte coalesced gathers of
+//                  the 656-byte rows (evict-first), exact dequantisation into
+//                  a double-buffered 64 x 576 bf16 K ring (128-byte swizzled,
+//                  K-major; the same tile read MN-major is V), Q loads;
+//       warp 8     one lane issues the MMAs and commits; the warp owns TMEM.
+//   * Order of the MMAs: S(t+1) is issued before PV(t), so the tensor core
+//     computes the next scores while the softmax warps work on the current
+//     ones.
+//   * The producers run a three-stage software pipeline across tiles: the
+//     indices of tile t+2 and the block-table entries of tile t+1 are loaded
+//     while tile t is dequantised, and the rows of tile t+1 right after, so
+//     the dependent loads index -> block table -> row never stall a tile.
+//   * TMEM (512 columns): O = 64 x 512 fp32 in columns [0, 256), its two
+//     256-wide halves in the lower and upper 16 lanes of each sub-partition
+//     (an M = 64 accumulator uses 16 lanes per sub-partition); S double
+//     buffer in columns [256, 320) and [320, 384), lanes 0-15.
+//   * Online softmax in base 2.  The running max used for P only moves when a
+//     tile's max exceeds it by more than 2^8 (then O and l are rescaled), so
+//     P <= 256 and rescales are rare; lse = (m + log2 l) ln 2 at the end.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include <cstdint>
+#include <cstring>
 
 #include "sm100.cuh"
 #include "splitkv_mla.h"
@@ -46,35 +61,54 @@ namespace {
 
 constexpr int kRows = 64;              // index slots per tile
 constexpr int kHeads = 64;             // heads per CTA (MMA M)
-constexpr int kThreads = 256;
+constexpr int kThreads = 288;          // 4 softmax + 4 producer warps + 1 MMA warp
+constexpr int kMmaWarp = 8;
 constexpr int kKBlocks = 9;            // 576 / 64 bf16 per 128-byte swizzle line
 constexpr int kAtom = kRows * 128;     // bytes of one 64-row x 128-byte column block
-constexpr int kQBytes = kKBlocks * kAtom;
-constexpr int kKBytes = kKBlocks * kAtom;
+constexpr int kTileBytes = kKBlocks * kAtom;
 constexpr int kPBytes = kAtom;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kOCol = 0;          // O: columns [0, 256), halves at lane offsets 0 / 16
-constexpr uint32_t kSCol = 256;        // S: columns [256, 320), lanes 0-15 of each sub-partition
+constexpr uint32_t kOCol = 0;
+constexpr uint32_t kSCol = 256;        // S buffer s at kSCol + 64 s
+constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no legitimate wait comes close
 
-struct __align__(16) SmemTail {
-  int64_t row_off[kRows];   // byte offset of each gathered row in the cache, -1 if invalid
-  uint64_t bar_s;           // S MMA complete
-  uint64_t bar_o;           // PV MMA complete
+struct __align__(16) Tail {
+  uint64_t kfull[2];   // K tile s written (producers of both CTAs of a pair)
+  uint64_t kempty[2];  // K tile s consumed by PV (both CTAs of a pair)
+  uint64_t sfull[2];   // S buffer s computed
+  uint64_t pfull;      // P written and O rescaled
+  uint64_t ofree;      // PV complete
+  uint64_t odrain;     // epilogue read O
+  uint64_t qfull;      // Q tile loaded
+  uint64_t qfree;      // last S of a request complete: sQ reusable
   uint32_t tmem_base;
-  int32_t abort_flag;
+  int32_t abort;
+  uint8_t vmask[2][8];  // per K buffer: bit k of byte i = row 8i+k holds a valid slot
 };
 
-constexpr int kSmemBytes = kQBytes + kKBytes + kPBytes + (int)sizeof(SmemTail) + 1024;
+constexpr int kOffQ = 0;
+constexpr int kOffK = kTileBytes;
+constexpr int kOffP = 3 * kTileBytes;
+constexpr int kOffTail = kOffP + kPBytes;
+constexpr int kSmemBytes = kOffTail + (int)sizeof(Tail) + 1024;
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk16) {
-  // byte offset of 16-byte chunk `chunk16` (0..7) of `row` inside one column block
   return (uint32_t)(row * 128 + ((chunk16 ^ (row & 7)) << 4));
 }
 
 __device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
-// 16 e4m3 values (one 16-byte chunk) -> 16 bf16 = bf16(float(e4m3) * scale).
+// 2^x on the special-function unit (P is rounded to bf16 right after).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 16 e4m3 values (one 16-byte chunk) -> 16 bf16 = bf16(float(e4m3) * scale):
+// hardware e4m3x2 -> f16x2 converts (exact), f16 -> f32 (exact), a
+// round-to-nearest f32 multiply, then round-to-nearest-even to bf16.
 __device__ __forceinline__ void dequant16(const uint4& raw, float scale, uint4& lo, uint4& hi) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
   uint32_t out[8];
@@ -96,40 +130,77 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
                : "memory");
 }
 
-__device__ __forceinline__ uint4 ldg_v4(const void* p) {
-  return __ldg(reinterpret_cast<const uint4*>(p));
+__device__ __forceinline__ void st_shared_u8(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u8 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+
+__device__ __forceinline__ void st_cluster_u8(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u8 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint64_t ld_shared_u64(uint32_t addr) {
+  uint64_t v;
+  asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+
+// Walks a part's (request, tile) range one round at a time (a tile has
+// `rounds` rounds of row loading), without any division in the loop.
+struct Cursor {
+  int r, t, q;
+  __device__ __forceinline__ void advance(int n, int rounds) {
+    if (++q == rounds) {
+      q = 0;
+      if (++t == n) {
+        t = 0;
+        ++r;
+      }
+    }
+  }
+};
 
 }  // namespace
 
+template <bool kPair>
 __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kQBytes;
-  uint8_t* sP = sK + kKBytes;
-  SmemTail* tail = reinterpret_cast<SmemTail*>(sP + kPBytes);
-  const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aP = smem_u32(sP);
+  Tail* tail = reinterpret_cast<Tail*>(smem + kOffTail);
+  const uint32_t aQ = smem_u32(smem + kOffQ);
+  const uint32_t aK0 = smem_u32(smem + kOffK);
+  const uint32_t aP = smem_u32(smem + kOffP);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int part = blockIdx.x;
-  const int hg = blockIdx.y;                       // head group: heads [64*hg, 64*hg + 64)
+  const uint32_t crank = kPair ? cluster_ctarank() : 0u;
+  const int hg = kPair ? (int)crank : (int)blockIdx.y;      // head group: heads [64*hg, 64*hg + 64)
   const int heads_here = min(kHeads, p.h_q - kHeads * hg);
+  const uint32_t peer = crank ^ 1u;
 
   if (tid == 0) {
-    mbar_init(&tail->bar_s, 1);
-    mbar_init(&tail->bar_o, 1);
-    tail->abort_flag = 0;
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&tail->kfull[s], kPair ? 8 : 4);
+      mbar_init(&tail->kempty[s], kPair ? 2 : 1);
+      mbar_init(&tail->sfull[s], 1);
+    }
+    mbar_init(&tail->pfull, 128);
+    mbar_init(&tail->ofree, 1);
+    mbar_init(&tail->odrain, 128);
+    mbar_init(&tail->qfull, 128);
+    mbar_init(&tail->qfree, 1);
+    tail->abort = 0;
     fence_mbarrier_init();
   }
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&tail->tmem_base, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
+  if (kPair) cluster_sync();       // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = tail->tmem_base;
 
@@ -149,277 +220,452 @@ __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVP
       empty = true;
     }
   }
+  const int n = p.n_tiles;
+  const int64_t g0 = empty ? 0 : (int64_t)m0.x * n + m0.y;
+  const int64_t g1 = empty ? 0 : (int64_t)m0.z * n + m0.w;
+  const int64_t ntile = g1 - g0;
 
-  uint32_t phase_s = 0, phase_o = 0;
-  const uint32_t idesc_s = idesc_bf16_f32(kHeads, kRows, false);
-  const uint32_t idesc_pv = idesc_bf16_f32(kHeads, 256, true);
-  const float scale_log2 = p.scale_log2;
+  if (warp >= 4 && warp < 8) {
+    // ======================= producers =====================================
+    // A warp owns 8 rows of a tile per round: one round per tile in the
+    // two-CTA form (32 rows per CTA), two rounds in the single-CTA form.
+    // Rounds are software-pipelined: the index of round R+2 and the
+    // block-table entry of round R+1 are loaded before round R is
+    // dequantised, and the rows of round R+1 right after it.  The loop body
+    // is kept small (one copy of each stage): the roles share the SM's
+    // instruction caches.
+    const int pw = warp - 4;
+    const int ptid = tid - 128;
+    const uint64_t pol = l2_evict_first_policy();
+    constexpr int kRounds = kPair ? 1 : 2;
+    const int64_t nround = ntile * kRounds;
+    // Stores: lane l writes the two 16-byte halves of its 32-byte output in
+    // an order that puts the 8 lanes of a quarter-warp on 8 distinct bank
+    // groups (lanes with bit 2 set start with the upper half).
+    const int kb = lane >> 2;
+    const int swap = (lane >> 2) & 1;
+    const int c_first = 2 * (lane & 3) + swap;
+    const int c_second = 2 * (lane & 3) + 1 - swap;
+    auto first_row = [&](int q) -> int { return kPair ? (32 * (int)crank + 8 * pw) : (32 * q + 8 * pw); };
+    Cursor ca{m0.x, m0.y, 0}, cb = ca, cf = ca;   // rounds R+2 (stage A), R+1 (stage B), R (fill)
+    int64_t jf = 0;                                // tile index of round R
 
-  // softmax row owned by this thread (warps 0-3, lanes 0-15)
-  const bool softmax_warp = warp < 4;
-  const int my_head = 16 * (warp & 3) + (lane & 15);   // row of the CTA's 64-head tile
-  const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
-
-  int r = m0.x, tile = m0.y;
-  const int end_r = m0.z, end_tile = m0.w;
-  bool first_req = true;
-  bool aborted = false;
-
-  while (!empty && !aborted && (r < end_r || (r == end_r && tile < end_tile))) {
-    const int tb = tile;
-    const int te = (r == end_r) ? end_tile : p.n_tiles;
-    const int ns_r = p.num_splits[r], ns_r1 = p.num_splits[r + 1];
-    const int slot = first_req ? m1.x : ns_r;
-    const int nsplit = ns_r1 - ns_r;
-    if (ns_r < 0 || ns_r1 > p.max_splits || nsplit < 1 || slot < ns_r || slot >= ns_r1) {
-      if (tid == 0) report_status(p.status, kStatusBadSchedule);
-      break;
+    int idx_a = -1, sl_a = 0;    // round R+2 (lanes 0-7)
+    int idx_b = -1, sl_b = 0;    // round R+1
+    int row_c = -1;              // round R: cache row of lane 0-7's slot, -1 if invalid
+    uint4 lat[8], rp[2];
+    float sc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      lat[k] = make_uint4(0u, 0u, 0u, 0u);
+      sc[k] = 0.f;
     }
-    const int b = r / p.s_q;
-    const int seqlen = p.seqlens[b];
-    const int32_t* bt = p.block_table + (size_t)b * p.max_blocks;
-    const int32_t* idx_row = p.indices + (size_t)r * p.topk;
+    rp[0] = rp[1] = make_uint4(0u, 0u, 0u, 0u);
 
-    // ---- Q tile: rows = heads of this group, zero rows past h_q ----------
-    {
-      const __nv_bfloat16* qsrc = p.q + ((size_t)r * p.h_q + (size_t)kHeads * hg) * 576;
-      for (int i = tid; i < kHeads * 72; i += kThreads) {
-        const int row = i / 72, ch = i % 72;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (row < heads_here) v = ldg_v4(qsrc + (size_t)row * 576 + ch * 8);
-        st_shared_v4(aQ + (ch >> 3) * kAtom + swz(row, ch & 7), v);
-      }
-    }
-
-    float m_run = -INFINITY, l_run = 0.f;   // base-2 running max and denominator
-
-    for (int t = tb; t < te && !aborted; ++t) {
-      // ---- indices -> cache row offsets -----------------------------------
-      if (tid < kRows) {
-        const int j = t * kRows + tid;
-        const int idx = (j < p.topk) ? idx_row[j] : -1;
-        int64_t off = -1;
-        if (idx >= 0 && idx < seqlen) {
-          const int blk = idx >> 6;
-          if (blk < p.max_blocks) {
-            const int64_t phys = bt[blk];
-            if (phys >= 0 && phys < p.num_blocks) off = (phys * 64 + (idx & 63)) * 656;
-            else report_status(p.status, kStatusBadBlockTable);
-          } else {
-            report_status(p.status, kStatusBadBlockTable);
-          }
-        }
-        tail->row_off[tid] = off;
-      }
-      __syncthreads();
-
-      // ---- gather + dequantise: warp w takes rows w, w+8, ...; lane = 16-byte chunk
-      {
-        uint4 raw[8];
-        float sc[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int64_t off = tail->row_off[warp + 8 * i];
-          raw[i] = make_uint4(0u, 0u, 0u, 0u);
-          sc[i] = 0.f;
-          if (off >= 0) {
-            raw[i] = ldg_v4(p.kv + off + 16 * lane);
-            sc[i] = __ldg(reinterpret_cast<const float*>(p.kv + off + 512) + (lane >> 3));
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int row = warp + 8 * i;
-          uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-          if (tail->row_off[row] >= 0) dequant16(raw[i], sc[i], lo, hi);
-          const uint32_t base = aK + (lane >> 2) * kAtom;
-          st_shared_v4(base + swz(row, 2 * (lane & 3)), lo);
-          st_shared_v4(base + swz(row, 2 * (lane & 3) + 1), hi);
-        }
-        // RoPE: 64 rows x 8 chunks of 16 bytes, copied into column block 8
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int c = tid + kThreads * k;
-          const int row = c >> 3, ch = c & 7;
-          const int64_t off = tail->row_off[row];
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (off >= 0) v = ldg_v4(p.kv + off + 528 + 16 * ch);
-          st_shared_v4(aK + 8 * kAtom + swz(row, ch), v);
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncthreads();
-
-      // ---- S = Q K^T -----------------------------------------------------
-      if (tid == 0) {
-        tc_fence_after();
+    int req_ord = -1;
+    bool ok = true;
 #pragma unroll 1
-        for (int kk = 0; kk < 36; ++kk) {
-          const uint32_t koff = (kk >> 2) * kAtom + (kk & 3) * 32;
-          mma_bf16_ss(tmem + kSCol, smem_desc_sw128(aQ + koff, 16, 1024), smem_desc_sw128(aK + koff, 16, 1024),
-                      idesc_s, kk > 0);
-        }
-        mma_commit(&tail->bar_s);
+    for (int64_t R = -2; R < nround && ok; ++R) {
+      // ---- stage A: index and request length of round R+2 -----------------
+      if (R + 2 < nround) {
+        const int slot = ca.t * kRows + first_row(ca.q) + lane;
+        idx_a = -1;
+        sl_a = 0;
+        ldg_s32_if(idx_a, p.indices + (size_t)ca.r * p.topk + slot, lane < 8 && slot < p.topk);
+        ldg_s32_if(sl_a, p.seqlens + ca.r / p.s_q, lane < 8);
+        ca.advance(n, kRounds);
       }
-      {
-        const bool ok = mbar_wait_bounded(&tail->bar_s, phase_s, kWaitLimitNs, p.status);
-        phase_s ^= 1;
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
+      // ---- stage B: block-table entry of round R+1 -------------------------
+      int phys_b = -1;
+      if (R + 1 >= 0 && R + 1 < nround) {
+        const bool valid = lane < 8 && idx_b >= 0 && idx_b < sl_b;
+        const int blk = idx_b >> 6;
+        if (valid && blk >= p.max_blocks) report_status(p.status, kStatusBadBlockTable);
+        ldg_s32_if(phys_b, p.block_table + (size_t)(cb.r / p.s_q) * p.max_blocks + blk,
+                   valid && blk < p.max_blocks);
+        cb.advance(n, kRounds);
       }
-      tc_fence_after();
-
-      // ---- online softmax (warps 0-3) ------------------------------------
-      if (softmax_warp) {
-        uint32_t s_lo[32], s_hi[32];
-        tmem_ld32(tmem + t_lane + kSCol, s_lo);
-        tmem_ld32(tmem + t_lane + kSCol + 32, s_hi);
-        tmem_wait_ld();
-        uint32_t s_raw[64];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          s_raw[j] = s_lo[j];
-          s_raw[32 + j] = s_hi[j];
-        }
-        float alpha = 1.f;
-        if (lane < 16) {
-          float mt = -INFINITY;
-#pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            float s = __uint_as_float(s_raw[j]) * scale_log2;
-            s = (tail->row_off[j] >= 0) ? s : -INFINITY;
-            s_raw[j] = __float_as_uint(s);
-            mt = fmaxf(mt, s);
-          }
-          const float m_new = fmaxf(m_run, mt);
-          uint32_t pw[32];
-          float psum = 0.f;
-          if (m_new == -INFINITY) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) pw[j] = 0u;
-          } else {
-            alpha = exp2f(m_run - m_new);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float p0 = exp2f(__uint_as_float(s_raw[2 * j]) - m_new);
-              const float p1 = exp2f(__uint_as_float(s_raw[2 * j + 1]) - m_new);
-              __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-              const float2 pr = __bfloat1622float2(pb);
-              psum += pr.x + pr.y;
-              pw[j] = bf162_bits(pb);
+      // ---- dequantise and store round R ------------------------------------
+      if (R >= 0) {
+        const int64_t j = jf;
+        const int q = cf.q;
+        const bool tile_first = (j == 0) || (cf.t == 0);
+        const int s = (int)(j & 1);
+        const uint32_t aK = aK0 + (uint32_t)s * kTileBytes;
+        const uint32_t aKr = kPair ? mapa_shared(aK, peer) : 0u;      // the peer's copy of this slot
+        if (q == 0) {
+          if (tile_first) {
+            ++req_ord;
+            if (req_ord > 0 &&
+                !mbar_wait_bounded_warp(&tail->qfree, (uint32_t)((req_ord - 1) & 1), kWaitLimitNs, p.status)) {
+              ok = false;
+              break;
             }
-            m_run = m_new;
-          }
-          l_run = l_run * alpha + psum;
-          // P row (64 bf16 = 8 chunks) -> K-major swizzled A operand
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            st_shared_v4(aP + swz(my_head, c), make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]));
-        }
-        // rescale the running output when the max moved (O exists after the first tile)
-        alpha = __shfl_sync(0xffffffffu, alpha, lane & 15);
-        const bool need = __any_sync(0xffffffffu, alpha != 1.f) && (t > tb);
-        if (need) {
+            const __nv_bfloat16* qsrc = p.q + ((size_t)cf.r * p.h_q + (size_t)kHeads * hg) * 576;
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem + t_lane + kOCol + 32 * c, o);
-            tmem_wait_ld();
+            for (int i0 = ptid; i0 < kHeads * 72; i0 += 128 * 6) {
+              uint4 v[6];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tmem_st32(tmem + t_lane + kOCol + 32 * c, o);
+              for (int u = 0; u < 6; ++u) {
+                const int i = i0 + 128 * u;
+                const bool live = i < kHeads * 72 && i / 72 < heads_here;
+                v[u] = make_uint4(0u, 0u, 0u, 0u);
+                ldg_v4_if(v[u], qsrc + (live ? (size_t)(i / 72) * 576 + (i % 72) * 8 : 0), live);
+              }
+#pragma unroll
+              for (int u = 0; u < 6; ++u) {
+                const int i = i0 + 128 * u;
+                if (i < kHeads * 72) st_shared_v4(aQ + ((i % 72) >> 3) * kAtom + swz(i / 72, (i % 72) & 7), v[u]);
+              }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&tail->qfull);
           }
-          tmem_wait_st();
+          // the ring slot is free once PV of tile j-2 finished in every CTA of the cluster
+          if (!mbar_wait_bounded_warp(&tail->kempty[s], (uint32_t)(((j >> 1) & 1) ^ 1), kWaitLimitNs, p.status)) {
+            ok = false;
+            break;
+          }
+        }
+        const int rb = first_row(q);
+        const uint32_t vbits = __ballot_sync(0xffffffffu, row_c >= 0) & 0xFFu;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int row = rb + k;
+          uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+          if ((vbits >> k) & 1u) dequant16(lat[k], sc[k], lo, hi);
+          const uint32_t o0 = kb * kAtom + swz(row, c_first);
+          const uint32_t o1 = kb * kAtom + swz(row, c_second);
+          const uint4 v0 = swap ? hi : lo;
+          const uint4 v1 = swap ? lo : hi;
+          st_shared_v4(aK + o0, v0);
+          st_shared_v4(aK + o1, v1);
+          if (kPair) {
+            st_cluster_v4(aKr + o0, v0);
+            st_cluster_v4(aKr + o1, v1);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const uint32_t orp = 8 * kAtom + swz(rb + 4 * i + (lane >> 3), lane & 7);
+          st_shared_v4(aK + orp, rp[i]);
+          if (kPair) st_cluster_v4(aKr + orp, rp[i]);
+        }
+        if (lane == 0) {
+          const uint32_t va = smem_u32(&tail->vmask[s][rb >> 3]);
+          st_shared_u8(va, vbits);
+          if (kPair) st_cluster_u8(mapa_shared(va, peer), vbits);
+        }
+        cf.advance(n, kRounds);
+        if (cf.q == 0) ++jf;
+        if (q == kRounds - 1) {
+          if (kPair) fence_proxy_async_cluster();
+          else fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&tail->kfull[s]);
+            if (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&tail->kfull[s]), peer));
+          }
         }
       }
+      // ---- stage C: row loads of round R+1 ---------------------------------
+      if (R + 1 >= 0 && R + 1 < nround) {
+        row_c = -1;
+        if (phys_b >= p.num_blocks) report_status(p.status, kStatusBadBlockTable);
+        else if (phys_b >= 0) row_c = phys_b * 64 + (idx_b & 63);
+        // For every row, lane l takes latent bytes [16l, 16l+16) and the scale
+        // of its 128-value tile; the 8 x 8 RoPE chunks are spread two per
+        // lane (row l/8 and 4 + l/8, chunk l%8).
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rk = __shfl_sync(0xffffffffu, row_c, k);
+          const uint8_t* row = p.kv + (int64_t)max(rk, 0) * 656;
+          lat[k] = make_uint4(0u, 0u, 0u, 0u);
+          sc[k] = 0.f;
+          ldg_v4_evict_first_if(lat[k], row + 16 * lane, rk >= 0, pol);
+          ldg_f32_evict_first_if(sc[k], row + 512 + 4 * (lane >> 3), rk >= 0, pol);
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int rk = __shfl_sync(0xffffffffu, row_c, 4 * i + (lane >> 3));
+          rp[i] = make_uint4(0u, 0u, 0u, 0u);
+          ldg_v4_evict_first_if(rp[i], p.kv + (int64_t)max(rk, 0) * 656 + 528 + 16 * (lane & 7), rk >= 0, pol);
+        }
+      }
+      idx_b = idx_a;
+      sl_b = sl_a;
+    }
+    // Every arrive aimed at this CTA's ring barriers (the peer's multicast
+    // commits included) has landed before the CTA may exit: wait for the last
+    // completion of each ring slot that was used.
+    if (lane == 0) {
+      for (int64_t j = ntile; j < ntile + 2; ++j) {
+        if (j - 2 < 0) continue;
+        (void)mbar_wait_bounded(&tail->kempty[j & 1], (uint32_t)(((j >> 1) & 1) ^ 1), kWaitLimitNs, p.status);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ======================= MMA issuer ====================================
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(kHeads, kRows, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(kHeads, 256, true);
+      // Descriptors are built once; an MMA step only adds its byte offset >> 4
+      // to the start-address field (all addresses stay below 2^18).
+      const uint64_t dQ = smem_desc_sw128(aQ, 16, 1024);
+      const uint64_t dK0 = smem_desc_sw128(aK0, 16, 1024);
+      const uint64_t dP = smem_desc_sw128(aP, 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(aK0, kAtom, 1024);
+      int req_ord = -1;
+      int prev_req_ord = -1;
+      bool prev_first = false;
+      Cursor cm{m0.x, m0.y, 0};
+      // Iteration j issues S(j) and then PV(j-1): the next scores are computed
+      // while the softmax warps turn S(j-1) into P(j-1).
+#pragma unroll 1
+      for (int64_t j = 0; j <= ntile; ++j) {
+        const bool t_first = (j == 0) || (cm.t == 0);
+        const bool t_last = (j == ntile - 1) || (cm.t == n - 1);
+        if (j < ntile) {
+          const int s = (int)(j & 1);
+          if (t_first) {
+            ++req_ord;
+            if (!mbar_wait_bounded(&tail->qfull, (uint32_t)(req_ord & 1), kWaitLimitNs, p.status)) break;
+          }
+          if (!mbar_wait_bounded(&tail->kfull[s], (uint32_t)((j >> 1) & 1), kWaitLimitNs, p.status)) break;
+          tc_fence_after();
+          const uint64_t dK = dK0 + (uint64_t)(((uint32_t)s * kTileBytes) >> 4);
+          const uint32_t d_s = tmem + kSCol + 64 * s;
+#pragma unroll 4
+          for (int kk = 0; kk < 36; ++kk) {
+            const uint64_t koff = (uint64_t)((((kk >> 2) * kAtom) + (kk & 3) * 32) >> 4);
+            mma_bf16_ss(d_s, dQ + koff, dK + koff, idesc_s, kk > 0);
+          }
+          if (t_last) mma_commit(&tail->qfree);
+          mma_commit(&tail->sfull[s]);
+        }
+        if (j >= 1) {
+          const int64_t i = j - 1;
+          if (!mbar_wait_bounded(&tail->pfull, (uint32_t)(i & 1), kWaitLimitNs, p.status)) break;
+          if (prev_first && prev_req_ord > 0 &&
+              !mbar_wait_bounded(&tail->odrain, (uint32_t)((prev_req_ord - 1) & 1), kWaitLimitNs, p.status))
+            break;
+          tc_fence_after();
+          const uint64_t dV = dV0 + (uint64_t)(((uint32_t)(i & 1) * kTileBytes) >> 4);
+#pragma unroll 1
+          for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+              mma_bf16_ss(tmem + kOCol + ((uint32_t)(16 * hh) << 16), dP + (uint64_t)((ks * 32) >> 4),
+                          dV + (uint64_t)(((4 * hh) * kAtom + ks * 16 * 128) >> 4), idesc_pv,
+                          (ks > 0 || !prev_first) ? 1u : 0u);
+          }
+          if (kPair) mma_commit_multicast(&tail->kempty[i & 1], (uint16_t)0x3);
+          else mma_commit(&tail->kempty[i & 1]);
+          mma_commit(&tail->ofree);
+        }
+        if (j < ntile) {
+          prev_first = t_first;
+          prev_req_ord = req_ord;
+          cm.advance(n, 1);
+        }
+      }
+      // the last request's qfree arrive lands before the CTA may exit
+      if (ntile > 0) (void)mbar_wait_bounded(&tail->qfree, (uint32_t)(req_ord & 1), kWaitLimitNs, p.status);
+    }
+  } else {
+    // ======================= softmax / epilogue (warps 0-3) =================
+    // S is read from TMEM in two 32-column halves, twice: once for the row
+    // max, once for P (keeping the code and the register footprint small).
+    const int my_head = 16 * warp + (lane & 15);
+    const uint32_t t_lane = (uint32_t)(32 * warp) << 16;
+    const float scale_log2 = p.scale_log2;
+    float m_used = -INFINITY, l_run = 0.f;
+    int req_ord = -1;
+    int slot = 0, nsplit = 1;
+    bool req_ok = true;
+    Cursor cx{m0.x, m0.y, 0};
+#pragma unroll 1
+    for (int64_t j = 0; j < ntile; ++j, cx.advance(n, 1)) {
+      struct {
+        int r;
+        bool first, last;
+      } tp{cx.r, (j == 0) || (cx.t == 0), (j == ntile - 1) || (cx.t == n - 1)};
+      const int s = (int)(j & 1);
+      const uint32_t ph = (uint32_t)((j >> 1) & 1);
+      if (tp.first) {
+        ++req_ord;
+        m_used = -INFINITY;
+        l_run = 0.f;
+        const int ns_r = p.num_splits[tp.r], ns_r1 = p.num_splits[tp.r + 1];
+        slot = (req_ord == 0) ? m1.x : ns_r;
+        nsplit = ns_r1 - ns_r;
+        req_ok = !(ns_r < 0 || ns_r1 > p.max_splits || nsplit < 1 || slot < ns_r || slot >= ns_r1);
+        if (!req_ok && tid == 0) report_status(p.status, kStatusBadSchedule);
+      }
+      if (!mbar_wait_bounded_warp(&tail->sfull[s], ph, kWaitLimitNs, p.status)) break;
+      if (!mbar_wait_bounded_warp(&tail->kfull[s], ph, kWaitLimitNs, p.status)) break;
+      tc_fence_after();
+      const uint64_t vm = ld_shared_u64(smem_u32(&tail->vmask[s][0]));
+      const uint32_t t_s = tmem + t_lane + kSCol + 64 * s;
+      float mt = -INFINITY;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * h, sr);
+        tmem_wait_ld();
+        const uint32_t vh = (uint32_t)(vm >> (32 * h));
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if ((vh >> c) & 1u) mt = fmaxf(mt, __uint_as_float(sr[c]));
+      }
+      float alpha = 1.f;
+      if (lane < 16) {
+        mt = (mt == -INFINITY) ? -INFINITY : mt * scale_log2;
+        if (mt > m_used + kRescaleLog2) {
+          alpha = fast_exp2(m_used - mt);     // 0 when nothing was valid before
+          l_run *= alpha;
+          m_used = mt;
+        }
+      }
+      // PV of the previous tile must be done before P is overwritten or O rescaled.
+      if (j >= 1 && !mbar_wait_bounded_warp(&tail->ofree, (uint32_t)((j - 1) & 1), kWaitLimitNs, p.status)) break;
+      tc_fence_after();
+      alpha = __shfl_sync(0xffffffffu, alpha, lane & 15);
+      if (!tp.first && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + t_lane + kOCol + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+          tmem_st32(tmem + t_lane + kOCol + 32 * c, o);
+        }
+        tmem_wait_st();
+      }
+      // P = 2^(s * scale_log2 - m) for valid slots (0 otherwise), rounded to bf16
+      const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
+      float psum = 0.f;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * h, sr);
+        tmem_wait_ld();
+        const uint32_t vh = (uint32_t)(vm >> (32 * h));
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float p0 = ((vh >> (2 * c)) & 1u) ? fast_exp2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, neg_m)) : 0.f;
+          const float p1 =
+              ((vh >> (2 * c + 1)) & 1u) ? fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, neg_m)) : 0.f;
+          psum += p0 + p1;
+          pk[c] = bf162_bits(__floats2bfloat162_rn(p0, p1));
+        }
+        if (lane < 16) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            st_shared_v4(aP + swz(my_head, 4 * h + c), make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
+        }
+      }
+      if (m_used != -INFINITY) l_run += psum;
       fence_proxy_async_smem();
       tc_fence_before();
-      __syncthreads();
+      mbar_arrive(&tail->pfull);
 
-      // ---- O += P V ------------------------------------------------------
-      if (tid == 0) {
+      if (tp.last) {
+        if (!mbar_wait_bounded_warp(&tail->ofree, (uint32_t)(j & 1), kWaitLimitNs, p.status)) break;
         tc_fence_after();
+        const float l_me = __shfl_sync(0xffffffffu, l_run, lane & 15);
+        const float m_me = __shfl_sync(0xffffffffu, m_used, lane & 15);
+        const int half = lane >> 4;
+        const int head = kHeads * hg + my_head;
+        const bool live = req_ok && (my_head < heads_here);
+        const float inv_l = (l_me > 0.f) ? 1.f / l_me : 0.f;
+        const float lse_val = (l_me > 0.f) ? (m_me + log2f(l_me)) * 0.69314718055994531f : -INFINITY;
 #pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t a_desc = smem_desc_sw128(aP + ks * 32, 16, 1024);
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            const uint64_t b_desc = smem_desc_sw128(aK + (4 * hh) * kAtom + ks * 16 * 128, kAtom, 1024);
-            mma_bf16_ss(tmem + kOCol + ((uint32_t)(16 * hh) << 16), a_desc, b_desc, idesc_pv,
-                        (ks > 0 || t > tb) ? 1u : 0u);
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[32];
+          __syncwarp();
+          tmem_ld32(tmem + t_lane + kOCol + 32 * c, o);
+          tmem_wait_ld();
+          const int col = half * 256 + 32 * c;
+          if (!live) {
+          } else if (nsplit == 1) {
+            __nv_bfloat16* dst = p.o + ((size_t)tp.r * p.h_q + head) * 512 + col;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 w;
+              w.x = bf162_bits(__floats2bfloat162_rn(__uint_as_float(o[8 * v + 0]) * inv_l,
+                                                     __uint_as_float(o[8 * v + 1]) * inv_l));
+              w.y = bf162_bits(__floats2bfloat162_rn(__uint_as_float(o[8 * v + 2]) * inv_l,
+                                                     __uint_as_float(o[8 * v + 3]) * inv_l));
+              w.z = bf162_bits(__floats2bfloat162_rn(__uint_as_float(o[8 * v + 4]) * inv_l,
+                                                     __uint_as_float(o[8 * v + 5]) * inv_l));
+              w.w = bf162_bits(__floats2bfloat162_rn(__uint_as_float(o[8 * v + 6]) * inv_l,
+                                                     __uint_as_float(o[8 * v + 7]) * inv_l));
+              reinterpret_cast<uint4*>(dst)[v] = w;
+            }
+          } else {
+            float* dst = p.o_accum + ((size_t)slot * p.h_q + head) * 512 + col;
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              reinterpret_cast<float4*>(dst)[v] =
+                  make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                              __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
           }
         }
-        mma_commit(&tail->bar_o);
-      }
-      {
-        const bool ok = mbar_wait_bounded(&tail->bar_o, phase_o, kWaitLimitNs, p.status);
-        phase_o ^= 1;
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-      }
-      tc_fence_after();
-    }
-    if (aborted) break;
-
-    // ---- epilogue: normalise and write (warps 0-3) ------------------------
-    if (softmax_warp) {
-      const float l_me = __shfl_sync(0xffffffffu, l_run, lane & 15);
-      const float m_me = __shfl_sync(0xffffffffu, m_run, lane & 15);
-      const int half = lane >> 4;
-      const int head = kHeads * hg + my_head;
-      const bool live = my_head < heads_here;
-      const float inv_l = (l_me > 0.f) ? 1.f / l_me : 0.f;
-      const float lse_val = (l_me > 0.f) ? (m_me + log2f(l_me)) * 0.69314718055994531f : -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t o[32];
-        __syncwarp();
-        tmem_ld32(tmem + t_lane + kOCol + 32 * c, o);
-        tmem_wait_ld();
-        const int col = half * 256 + 32 * c;
-        if (!live) {
-        } else if (nsplit == 1) {
-          __nv_bfloat16* dst = p.o + ((size_t)r * p.h_q + head) * 512 + col;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = bf162_bits(__floats2bfloat162_rn(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l));
-            w.y = bf162_bits(__floats2bfloat162_rn(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l));
-            w.z = bf162_bits(__floats2bfloat162_rn(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l));
-            w.w = bf162_bits(__floats2bfloat162_rn(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l));
-            reinterpret_cast<uint4*>(dst)[v] = w;
-          }
-        } else {
-          float* dst = p.o_accum + ((size_t)slot * p.h_q + head) * 512 + col;
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            reinterpret_cast<float4*>(dst)[v] =
-                make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
-                            __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+        if (live && lane < 16) {
+          if (nsplit == 1) p.lse[(size_t)tp.r * p.h_q + head] = lse_val;
+          else p.lse_accum[(size_t)slot * p.h_q + head] = lse_val;
         }
-      }
-      if (live && lane < 16) {
-        if (nsplit == 1) p.lse[(size_t)r * p.h_q + head] = lse_val;
-        else p.lse_accum[(size_t)slot * p.h_q + head] = lse_val;
+        tc_fence_before();
+        mbar_arrive(&tail->odrain);
       }
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    r += 1;
-    tile = 0;
-    first_req = false;
   }
 
   pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (kPair) cluster_sync();
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
 }
 
 int splitkv_smem_bytes() { return kSmemBytes; }
+
+// Host launcher shared by the entry points: picks the single-CTA or the
+// two-CTA cluster form and chains the launch to the previous kernel of the
+// stream with programmatic dependent launch.
+cudaError_t launch_splitkv(const SplitKVParams& p, cudaStream_t stream) {
+  const bool pair = p.h_q > kHeads;
+  cudaLaunchAttribute attrs[2];
+  std::memset(attrs, 0, sizeof(attrs));
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  attrs[1].id = cudaLaunchAttributeClusterDimension;
+  attrs[1].val.clusterDim.x = 1;
+  attrs[1].val.clusterDim.y = 2;
+  attrs[1].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(p.num_parts, pair ? 2 : 1);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attrs;
+  cfg.numAttrs = pair ? 2 : 1;
+  if (pair) return cudaLaunchKernelEx(&cfg, splitkv_mla_kernel<true>, p);
+  return cudaLaunchKernelEx(&cfg, splitkv_mla_kernel<false>, p);
+}
+
+cudaError_t configure_splitkv() {
+  cudaError_t e =
+      cudaFuncSetAttribute(splitkv_mla_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(splitkv_mla_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+}
 
 }  // namespace smla

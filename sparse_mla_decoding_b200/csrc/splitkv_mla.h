@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_runtime.h>
 
 #include <cstdint>
 
@@ -28,7 +29,12 @@ struct SplitKVParams {
   uint32_t* status;             // sticky status word
 };
 
-__global__ void splitkv_mla_kernel(const SplitKVParams p);
+// Dynamic shared memory of the split kernel, its one-time attribute set-up
+// (per device) and its launch (single CTA for <= 64 heads, a two-CTA cluster
+// for 128 heads; chained to the previous kernel with programmatic dependent
+// launch).
 int splitkv_smem_bytes();
+cudaError_t configure_splitkv();
+cudaError_t launch_splitkv(const SplitKVParams& p, cudaStream_t stream);
 
 }  // namespace smla

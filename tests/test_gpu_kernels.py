@@ -205,3 +205,47 @@ def test_bitwise_deterministic(smla, torch_cuda):
     o1, l1, _, _ = PU.run_gpu(hi, dev_inputs=d)
     o2, l2, _, _ = PU.run_gpu(hi, dev_inputs=d)
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_dequant_every_code_and_scale_range_is_exact(smla, torch_cuda):
+    """A single valid slot makes o equal its value row exactly, so o exposes the
+    dequantised latent values: every e4m3 code (NaN codes included) times
+    scales from subnormal to > 2^8 must equal bf16(float(e4m3) * scale)."""
+    torch = torch_cuda
+    scales = [1.0, 2.0 ** -20, 3.7e-3, 300.0, 2.0 ** -130, 0.0, 1.5e-38, 123.456]
+    rows = []
+    for r, sc0 in enumerate(scales):
+        row = np.zeros(656, np.uint8)
+        codes = (np.arange(512) * 7 + 37 * r) % 256
+        codes[(codes & 0x7F) == 0x7F] -= 1              # the NaN codes poison S as well: kept out here
+        row[:512] = codes
+        row[512:528] = np.array([sc0, scales[(r + 1) % len(scales)], scales[(r + 3) % len(scales)], 1.0],
+                                np.float32).view(np.uint8)
+        row[528:] = 0                                      # zero RoPE: the scores stay finite
+        rows.append(row)
+    n = len(rows)
+    cache = np.zeros((1, 64, 656), np.uint8)
+    cache[0, :n] = np.stack(rows)
+    q_bits = W._to_bf16_bits(np.random.default_rng(3).standard_normal((n, 1, 16, 576)).astype(np.float32) * 0.01)
+    idx = np.full((n, 1, 64), -1, np.int32)
+    for r in range(n):
+        idx[r, 0, 5] = r
+    w = W.Workload("codes", batch=n, s_q=1, h_q=16, topk=64, seed=0, seqlens=(64,) * n)
+    hi = PU.HostInputs(w, q_bits, cache, np.zeros((n, 1), np.int32), np.full(n, 64, np.int32), idx)
+    d = PU.to_device(hi)
+    import sparse_mla_decoding_b200 as m
+    sm, ns = m.get_mla_metadata(d["cache_seqlens"], 64, 16, s_q=1)
+    o, lse = m.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"], sm, ns)
+    o = o.float().cpu().numpy()
+    for r in range(n):
+        v = oracle.dequantize_row(cache[0, r])[:512]
+        got = o[r, 0]
+        assert np.array_equal(np.isnan(got), np.broadcast_to(np.isnan(v), got.shape)), f"row {r}: NaN pattern"
+        ok = ~np.isnan(v)
+        assert np.array_equal(got[:, ok], np.broadcast_to(v[ok], (16, ok.sum()))), f"row {r} (scale {scales[r]})"
+    # a NaN code in a valid row reaches every score of the token: its output is NaN
+    cache2 = cache.copy()
+    cache2[0, 0, 100] = 0x7F
+    d["kvcache"] = torch.from_numpy(cache2).cuda()
+    o2, _ = m.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"], sm, ns)
+    assert np.isnan(o2[0, 0].float().cpu().numpy()).all()
