@@ -76,6 +76,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test: true once the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // try_wait with a suspend-time hint: the thread sleeps until the phase
 // completes or about `hint_ns` nanoseconds pass, instead of spinning (a
 // spinning waiter occupies the shared-memory pipe the working warps need).
@@ -249,6 +262,25 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
 // releasing this thread's prior writes at cluster scope.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+
+// Arrive on a peer CTA's mbarrier and raise its expected transaction count by
+// `bytes` (the bytes that bulk copies from this CTA will complete on it).
+__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t remote_bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(remote_bar),
+               "r"(bytes)
+               : "memory");
+}
+
+// Bulk copy (copy engine, no multicast) of `bytes` from this CTA's shared
+// memory to a peer CTA's shared memory; the copy completes `bytes` of
+// transaction count on the peer's mbarrier.  Addresses 16-byte aligned, size a
+// multiple of 16; `dst` and `remote_bar` come from mapa.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t remote_bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst),
+               "r"(src), "r"(bytes), "r"(remote_bar)
+               : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_cluster() {

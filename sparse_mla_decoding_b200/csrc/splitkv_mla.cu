@@ -21,7 +21,9 @@
 // Design on B200:
 //   * A CTA owns 64 query heads of one request at a time (M = 64 of every
 //     tcgen05.mma).  128 heads run as a two-CTA cluster (one CTA per 64-head
-//     group) that shares the dequantised tiles over distributed shared memory;
+//     group) that shares the dequantised tiles over distributed shared memory
+//     (each CTA dequantises half of the rows, and the copy engine sends them
+//     to the peer with bulk shared-to-shared copies);
 //     16/32 heads are zero-padded to 64 in a single CTA.
 //   * Warp roles (288 threads):
 //       warps 0-3  softmax: online softmax over S in TMEM, P to shared memory,
@@ -31,9 +33,10 @@
 //                  a double-buffered 64 x 576 bf16 K ring (128-byte swizzled,
 //                  K-major; the same tile read MN-major is V), Q loads;
 //       warp 8     one lane issues the MMAs and commits; the warp owns TMEM.
-//   * Order of the MMAs: S(t+1) is issued before PV(t), so the tensor core
-//     computes the next scores while the softmax warps work on the current
-//     ones.
+//   * Order of the MMAs: S(t+1) and PV(t) are issued as their inputs become
+//     ready, so the tensor core computes the next scores while the softmax
+//     warps work on the current ones, and a late tile never delays the PV
+//     that frees a ring slot.
 //   * The producers run a three-stage software pipeline across tiles: the
 //     indices of tile t+2 and the block-table entries of tile t+1 are loaded
 //     while tile t is dequantised, and the rows of tile t+1 right after, so
@@ -72,6 +75,10 @@ constexpr uint32_t kOCol = 0;
 constexpr uint32_t kSCol = 256;        // S buffer s at kSCol + 64 s
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no legitimate wait comes close
+#ifndef SMLA_POLL_SLEEP_NS
+#define SMLA_POLL_SLEEP_NS 32
+#endif
+constexpr uint32_t kPollSleepNs = SMLA_POLL_SLEEP_NS;  // MMA issuer back-off between readiness polls
 
 struct __align__(16) Tail {
   uint64_t kfull[2];   // K tile s written (producers of both CTAs of a pair)
@@ -340,17 +347,9 @@ __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVP
           const uint4 v1 = swap ? lo : hi;
           st_shared_v4(aK + o0, v0);
           st_shared_v4(aK + o1, v1);
-          if (kPair) {
-            st_cluster_v4(aKr + o0, v0);
-            st_cluster_v4(aKr + o1, v1);
-          }
         }
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const uint32_t orp = 8 * kAtom + swz(rb + 4 * i + (lane >> 3), lane & 7);
-          st_shared_v4(aK + orp, rp[i]);
-          if (kPair) st_cluster_v4(aKr + orp, rp[i]);
-        }
+        for (int i = 0; i < 2; ++i) st_shared_v4(aK + 8 * kAtom + swz(rb + 4 * i + (lane >> 3), lane & 7), rp[i]);
         if (lane == 0) {
           const uint32_t va = smem_u32(&tail->vmask[s][rb >> 3]);
           st_shared_u8(va, vbits);
@@ -359,12 +358,19 @@ __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVP
         cf.advance(n, kRounds);
         if (cf.q == 0) ++jf;
         if (q == kRounds - 1) {
-          if (kPair) fence_proxy_async_cluster();
-          else fence_proxy_async_smem();
+          fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&tail->kfull[s]);
-            if (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&tail->kfull[s]), peer));
+          if (lane == 0) mbar_arrive(&tail->kfull[s]);
+          if (kPair) {
+            // The copy engine sends this warp's 8 rows (1 KB in each of the 9
+            // column blocks, same offsets) to the peer's slot; the peer's kfull
+            // counts the arrive and the 9 KB of completed copies.
+            const uint32_t rbar = mapa_shared(smem_u32(&tail->kfull[s]), peer);
+            if (lane == 0) mbar_arrive_expect_tx_cluster(rbar, kKBlocks * 8 * 128);
+            if (lane < kKBlocks) {
+              const uint32_t off = (uint32_t)(lane * kAtom + rb * 128);
+              bulk_copy_to_peer(aKr + off, aK + off, 8 * 128, rbar);
+            }
           }
         }
       }
@@ -419,50 +425,71 @@ __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVP
       int prev_req_ord = -1;
       bool prev_first = false;
       Cursor cm{m0.x, m0.y, 0};
-      // Iteration j issues S(j) and then PV(j-1): the next scores are computed
-      // while the softmax warps turn S(j-1) into P(j-1).
+      // Iteration j issues S(j) and PV(j-1), whichever has its inputs first:
+      // the next scores are computed while the softmax warps turn S(j-1) into
+      // P(j-1), and a late tile j does not hold back PV(j-1) (whose commit
+      // frees a ring slot for the producers).  Readiness is polled with
+      // non-blocking tests; each barrier polled here cannot complete a second
+      // phase before the MMA this loop issues next.
 #pragma unroll 1
       for (int64_t j = 0; j <= ntile; ++j) {
         const bool t_first = (j == 0) || (cm.t == 0);
         const bool t_last = (j == ntile - 1) || (cm.t == n - 1);
-        if (j < ntile) {
-          const int s = (int)(j & 1);
-          if (t_first) {
-            ++req_ord;
-            if (!mbar_wait_bounded(&tail->qfull, (uint32_t)(req_ord & 1), kWaitLimitNs, p.status)) break;
-          }
-          if (!mbar_wait_bounded(&tail->kfull[s], (uint32_t)((j >> 1) & 1), kWaitLimitNs, p.status)) break;
-          tc_fence_after();
-          const uint64_t dK = dK0 + (uint64_t)(((uint32_t)s * kTileBytes) >> 4);
-          const uint32_t d_s = tmem + kSCol + 64 * s;
+        bool need_s = j < ntile, need_pv = j >= 1;
+        if (need_s && t_first) ++req_ord;
+        const int s = (int)(j & 1);
+        const int64_t i = j - 1;
+        const bool wait_drain = need_pv && prev_first && prev_req_ord > 0;
+        uint64_t t0 = 0;
+        bool stalled = false;
+        while (need_s || need_pv) {
+          bool went = false;
+          if (need_s && mbar_test_wait(&tail->kfull[s], (uint32_t)((j >> 1) & 1)) &&
+              (!t_first || mbar_test_wait(&tail->qfull, (uint32_t)(req_ord & 1)))) {
+            tc_fence_after();
+            const uint64_t dK = dK0 + (uint64_t)(((uint32_t)s * kTileBytes) >> 4);
+            const uint32_t d_s = tmem + kSCol + 64 * s;
 #pragma unroll 4
-          for (int kk = 0; kk < 36; ++kk) {
-            const uint64_t koff = (uint64_t)((((kk >> 2) * kAtom) + (kk & 3) * 32) >> 4);
-            mma_bf16_ss(d_s, dQ + koff, dK + koff, idesc_s, kk > 0);
+            for (int kk = 0; kk < 36; ++kk) {
+              const uint64_t koff = (uint64_t)((((kk >> 2) * kAtom) + (kk & 3) * 32) >> 4);
+              mma_bf16_ss(d_s, dQ + koff, dK + koff, idesc_s, kk > 0);
+            }
+            if (t_last) mma_commit(&tail->qfree);
+            mma_commit(&tail->sfull[s]);
+            need_s = false;
+            went = true;
           }
-          if (t_last) mma_commit(&tail->qfree);
-          mma_commit(&tail->sfull[s]);
-        }
-        if (j >= 1) {
-          const int64_t i = j - 1;
-          if (!mbar_wait_bounded(&tail->pfull, (uint32_t)(i & 1), kWaitLimitNs, p.status)) break;
-          if (prev_first && prev_req_ord > 0 &&
-              !mbar_wait_bounded(&tail->odrain, (uint32_t)((prev_req_ord - 1) & 1), kWaitLimitNs, p.status))
-            break;
-          tc_fence_after();
-          const uint64_t dV = dV0 + (uint64_t)(((uint32_t)(i & 1) * kTileBytes) >> 4);
+          if (need_pv && mbar_test_wait(&tail->pfull, (uint32_t)(i & 1)) &&
+              (!wait_drain || mbar_test_wait(&tail->odrain, (uint32_t)((prev_req_ord - 1) & 1)))) {
+            tc_fence_after();
+            const uint64_t dV = dV0 + (uint64_t)(((uint32_t)(i & 1) * kTileBytes) >> 4);
 #pragma unroll 1
-          for (int ks = 0; ks < 4; ++ks) {
+            for (int ks = 0; ks < 4; ++ks) {
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-              mma_bf16_ss(tmem + kOCol + ((uint32_t)(16 * hh) << 16), dP + (uint64_t)((ks * 32) >> 4),
-                          dV + (uint64_t)(((4 * hh) * kAtom + ks * 16 * 128) >> 4), idesc_pv,
-                          (ks > 0 || !prev_first) ? 1u : 0u);
+              for (int hh = 0; hh < 2; ++hh)
+                mma_bf16_ss(tmem + kOCol + ((uint32_t)(16 * hh) << 16), dP + (uint64_t)((ks * 32) >> 4),
+                            dV + (uint64_t)(((4 * hh) * kAtom + ks * 16 * 128) >> 4), idesc_pv,
+                            (ks > 0 || !prev_first) ? 1u : 0u);
+            }
+            if (kPair) mma_commit_multicast(&tail->kempty[i & 1], (uint16_t)0x3);
+            else mma_commit(&tail->kempty[i & 1]);
+            mma_commit(&tail->ofree);
+            need_pv = false;
+            went = true;
           }
-          if (kPair) mma_commit_multicast(&tail->kempty[i & 1], (uint16_t)0x3);
-          else mma_commit(&tail->kempty[i & 1]);
-          mma_commit(&tail->ofree);
+          if (went) {
+            stalled = false;
+          } else if (!stalled) {
+            stalled = true;
+            t0 = global_timer_ns();
+          } else if (global_timer_ns() - t0 > kWaitLimitNs) {
+            report_status(p.status, kStatusTimeout);
+            break;
+          } else {
+            __nanosleep(kPollSleepNs);
+          }
         }
+        if (need_s || need_pv) break;
         if (j < ntile) {
           prev_first = t_first;
           prev_req_ord = req_ord;
