@@ -158,21 +158,28 @@ __device__ __forceinline__ void tc_fence_after() {
 // ---------------------------------------------------------------------------
 // tcgen05.mma, kind::f16 (bf16 x bf16 -> fp32), A and B from shared memory
 // ---------------------------------------------------------------------------
+// These are called by a whole converged warp: the descriptor arithmetic stays
+// warp-uniform and one lane picked by elect.sync issues the instruction.
+// Issuing from a single lane inside a divergent branch instead makes every
+// MMA wait on per-thread operand moves, which halves the M = 64 issue rate.
 __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
 // Arrive (once) on an mbarrier when every tcgen05 operation issued so far by
-// this thread has completed.
+// the elected thread has completed.  Whole warp, like the MMAs.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -221,6 +228,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
+}
+
+// The two 32-bit halves of that descriptor.  Every 128-byte-swizzled operand
+// with a 1024-byte stride shares the upper half, and a step along K or along a
+// tile only changes the 14-bit start field of the lower half (no carry while
+// shared addresses stay below 256 KB), so MMA blocks add literal offsets to a
+// base lower half.
+__device__ __forceinline__ uint32_t smem_desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint32_t smem_desc_hi_sw128(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
 }
 
 // Instruction descriptor for kind::f16 with bf16 inputs and fp32 accumulate:
@@ -292,13 +311,19 @@ __device__ __forceinline__ void cluster_sync() {
 }
 
 // tcgen05.commit that arrives on the mbarrier at the same shared-memory offset
-// in every CTA of `cta_mask`.
+// in every CTA of `cta_mask`.  Whole warp, one elected lane issues.
 __device__ __forceinline__ void mma_commit_multicast(uint64_t* bar, uint16_t cta_mask) {
   asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}" ::"r"(
           smem_u32(bar)),
       "h"(cta_mask)
       : "memory");
+}
+
+// Non-blocking test by a whole warp: every lane tests, lane 0's answer counts.
+__device__ __forceinline__ bool mbar_test_wait_warp(uint64_t* bar, uint32_t parity) {
+  return __shfl_sync(0xffffffffu, mbar_test_wait(bar, parity) ? 1u : 0u, 0) != 0;
 }
 
 // ---------------------------------------------------------------------------

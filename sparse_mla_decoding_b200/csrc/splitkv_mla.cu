@@ -32,7 +32,8 @@
 //                  the 656-byte rows (evict-first), exact dequantisation into
 //                  a double-buffered 64 x 576 bf16 K ring (128-byte swizzled,
 //                  K-major; the same tile read MN-major is V), Q loads;
-//       warp 8     one lane issues the MMAs and commits; the warp owns TMEM.
+//       warp 8     MMA issuer: the warp runs the issue loop, one elected lane
+//                  issues each MMA and commit; the warp owns TMEM.
 //   * Order of the MMAs: S(t+1) and PV(t) are issued as their inputs become
 //     ready, so the tensor core computes the next scores while the softmax
 //     warps work on the current ones, and a late tile never delays the PV
@@ -64,12 +65,19 @@ namespace {
 
 constexpr int kRows = 64;              // index slots per tile
 constexpr int kHeads = 64;             // heads per CTA (MMA M)
-constexpr int kThreads = 288;          // 4 softmax + 4 producer warps + 1 MMA warp
-constexpr int kMmaWarp = 8;
+constexpr int kProducerWarps = 8;
+constexpr int kMmaWarp = 4 + kProducerWarps;
+constexpr int kThreads = 32 * (kMmaWarp + 1);   // 4 softmax + 8 producer warps + 1 MMA warp = 416
+// Warps are spread over the 4 SM sub-partitions by index, so one of them
+// holds 4 of the 13 warps: registers are capped at 16384 / (4 x 32) = 128 per
+// thread (the launch bound below asks for that cap).
+constexpr int kRegCapThreads = 512;
 constexpr int kKBlocks = 9;            // 576 / 64 bf16 per 128-byte swizzle line
 constexpr int kAtom = kRows * 128;     // bytes of one 64-row x 128-byte column block
 constexpr int kTileBytes = kKBlocks * kAtom;
 constexpr int kPBytes = kAtom;
+static_assert(kAtom == 8192 && kKBlocks == 9, "the MMA blocks below encode 64-row column blocks as literal offsets");
+static_assert(3 * kTileBytes + kAtom < (1 << 18), "descriptor start fields are 14 bits of (address >> 4)");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = 0;
 constexpr uint32_t kSCol = 256;        // S buffer s at kSCol + 64 s
@@ -91,7 +99,7 @@ struct __align__(16) Tail {
   uint64_t qfree;      // last S of a request complete: sQ reusable
   uint32_t tmem_base;
   int32_t abort;
-  uint8_t vmask[2][8];  // per K buffer: bit k of byte i = row 8i+k holds a valid slot
+  uint8_t vmask[2][16];  // per K buffer: bit k of byte g = row 4g+k holds a valid slot
 };
 
 constexpr int kOffQ = 0;
@@ -105,6 +113,60 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk16) {
 }
 
 __device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
+
+// One S tile: 36 MMAs (9 column blocks x 4 K-steps of 16) of M = 64, N = 64,
+// issued by one elected lane of a converged warp.  Operands: D column, Q and
+// K descriptor lower halves, the shared upper half, the instruction
+// descriptor.  A K-step adds 32 bytes (2 in descriptor units) and a column
+// block kAtom = 8192 bytes (512).
+#define SMLA_S_STEP(kb, k4, acc)                                       \
+  "add.u32 la, %1, (" #kb "*512+" #k4 "*2);\n\t"                       \
+  "add.u32 lb, %2, (" #kb "*512+" #k4 "*2);\n\t"                       \
+  "mov.b64 da, {la, %3};\n\t"                                          \
+  "mov.b64 db, {lb, %3};\n\t"                                          \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, " acc ";\n\t"
+#define SMLA_S_BLOCK(kb) \
+  SMLA_S_STEP(kb, 0, "pt") SMLA_S_STEP(kb, 1, "pt") SMLA_S_STEP(kb, 2, "pt") SMLA_S_STEP(kb, 3, "pt")
+
+__device__ __forceinline__ void issue_s_tile(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo, uint32_t hi,
+                                             uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred e, pt, pf;\n\t.reg .b32 la, lb;\n\t.reg .b64 da, db;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 pt, 1, 0;\n\t"
+      "setp.eq.b32 pf, 1, 0;\n\t"
+      SMLA_S_STEP(0, 0, "pf") SMLA_S_STEP(0, 1, "pt") SMLA_S_STEP(0, 2, "pt") SMLA_S_STEP(0, 3, "pt")
+      SMLA_S_BLOCK(1) SMLA_S_BLOCK(2) SMLA_S_BLOCK(3) SMLA_S_BLOCK(4)
+      SMLA_S_BLOCK(5) SMLA_S_BLOCK(6) SMLA_S_BLOCK(7) SMLA_S_BLOCK(8)
+      "}" ::"r"(d_tmem), "r"(q_lo), "r"(k_lo), "r"(hi), "r"(idesc)
+      : "memory");
+}
+
+// One PV step set: O[:, 256 hh + (0..255)] += P[:, 16 ks + (0..15)] V[16 ks + (0..15), ...]
+// for ks = 0..3, hh = 0..1 (8 MMAs of M = 64, N = 256; V read MN-major from
+// the K tile).  A K-step of P adds 32 bytes (2); of V 16 rows x 128 bytes
+// (128); the second 256 columns of V start 4 column blocks later (2048).
+#define SMLA_PV_STEP(ks, hh, acc)                                      \
+  "add.u32 la, %2, (" #ks "*2);\n\t"                                   \
+  "add.u32 lb, %3, (" #hh "*2048+" #ks "*128);\n\t"                    \
+  "mov.b64 da, {la, %4};\n\t"                                          \
+  "mov.b64 db, {lb, %4};\n\t"                                          \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%" #hh "], da, db, %5, " acc ";\n\t"
+
+__device__ __forceinline__ void issue_pv_tile(uint32_t d_lo16, uint32_t d_hi16, uint32_t p_lo, uint32_t v_lo,
+                                              uint32_t hi, uint32_t idesc, uint32_t accumulate_first) {
+  asm volatile(
+      "{\n\t.reg .pred e, pt, pa;\n\t.reg .b32 la, lb;\n\t.reg .b64 da, db;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 pt, 1, 0;\n\t"
+      "setp.ne.b32 pa, %6, 0;\n\t"
+      SMLA_PV_STEP(0, 0, "pa") SMLA_PV_STEP(0, 1, "pa")
+      SMLA_PV_STEP(1, 0, "pt") SMLA_PV_STEP(1, 1, "pt")
+      SMLA_PV_STEP(2, 0, "pt") SMLA_PV_STEP(2, 1, "pt")
+      SMLA_PV_STEP(3, 0, "pt") SMLA_PV_STEP(3, 1, "pt")
+      "}" ::"r"(d_lo16), "r"(d_hi16), "r"(p_lo), "r"(v_lo), "r"(hi), "r"(idesc), "r"(accumulate_first)
+      : "memory");
+}
 
 // 2^x on the special-function unit (P is rounded to bf16 right after).
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -152,17 +214,22 @@ __device__ __forceinline__ uint64_t ld_shared_u64(uint32_t addr) {
 }
 
 
-// Walks a part's (request, tile) range one round at a time (a tile has
-// `rounds` rounds of row loading), without any division in the loop.
+// Eight bytes, each holding 4 bits in its low nibble -> 32 packed bits.
+__device__ __forceinline__ uint32_t nibbles_to_bits(uint64_t x) {
+  x = (x | (x >> 4)) & 0x00FF00FF00FF00FFull;
+  x = (x | (x >> 8)) & 0x0000FFFF0000FFFFull;
+  x = (x | (x >> 16)) & 0x00000000FFFFFFFFull;
+  return (uint32_t)x;
+}
+
+// Walks a part's (request, tile) range one tile at a time, without any
+// division in the loop.
 struct Cursor {
-  int r, t, q;
-  __device__ __forceinline__ void advance(int n, int rounds) {
-    if (++q == rounds) {
-      q = 0;
-      if (++t == n) {
-        t = 0;
-        ++r;
-      }
+  int r, t;
+  __device__ __forceinline__ void advance(int n) {
+    if (++t == n) {
+      t = 0;
+      ++r;
     }
   }
 };
@@ -170,7 +237,7 @@ struct Cursor {
 }  // namespace
 
 template <bool kPair>
-__global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVParams p) {
+__global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const SplitKVParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Tail* tail = reinterpret_cast<Tail*>(smem + kOffTail);
@@ -189,14 +256,14 @@ __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVP
 
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&tail->kfull[s], kPair ? 8 : 4);
+      mbar_init(&tail->kfull[s], kPair ? 2 * kProducerWarps : kProducerWarps);
       mbar_init(&tail->kempty[s], kPair ? 2 : 1);
       mbar_init(&tail->sfull[s], 1);
     }
     mbar_init(&tail->pfull, 128);
     mbar_init(&tail->ofree, 1);
     mbar_init(&tail->odrain, 128);
-    mbar_init(&tail->qfull, 128);
+    mbar_init(&tail->qfull, 32 * kProducerWarps);
     mbar_init(&tail->qfree, 1);
     tail->abort = 0;
     fence_mbarrier_init();
@@ -232,20 +299,21 @@ __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVP
   const int64_t g1 = empty ? 0 : (int64_t)m0.z * n + m0.w;
   const int64_t ntile = g1 - g0;
 
-  if (warp >= 4 && warp < 8) {
+  if (warp >= 4 && warp < 4 + kProducerWarps) {
     // ======================= producers =====================================
-    // A warp owns 8 rows of a tile per round: one round per tile in the
-    // two-CTA form (32 rows per CTA), two rounds in the single-CTA form.
-    // Rounds are software-pipelined: the index of round R+2 and the
-    // block-table entry of round R+1 are loaded before round R is
-    // dequantised, and the rows of round R+1 right after it.  The loop body
-    // is kept small (one copy of each stage): the roles share the SM's
-    // instruction caches.
+    // Warp pw owns kRPW consecutive rows of every tile: 8 in the single-CTA
+    // form, 4 in the two-CTA form (where a CTA dequantises 32 of the 64 rows
+    // and sends them to its peer).  Tiles are software-pipelined: the index
+    // of tile t+2 and the block-table entry of tile t+1 are loaded before
+    // tile t is dequantised, and the rows of tile t+1 right after it, so
+    // they are in flight while the warp waits for the next ring slot.  The
+    // loop body is kept small (one copy of each stage): the roles share the
+    // SM's instruction caches.
+    constexpr int kRPW = kPair ? 4 : 8;
     const int pw = warp - 4;
     const int ptid = tid - 128;
     const uint64_t pol = l2_evict_first_policy();
-    constexpr int kRounds = kPair ? 1 : 2;
-    const int64_t nround = ntile * kRounds;
+    const int rb = kPair ? (32 * (int)crank + kRPW * pw) : kRPW * pw;   // this warp's first row of a tile
     // Stores: lane l writes the two 16-byte halves of its 32-byte output in
     // an order that puts the 8 lanes of a quarter-warp on 8 distinct bank
     // groups (lanes with bit 2 set start with the upper half).
@@ -253,137 +321,130 @@ __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVP
     const int swap = (lane >> 2) & 1;
     const int c_first = 2 * (lane & 3) + swap;
     const int c_second = 2 * (lane & 3) + 1 - swap;
-    auto first_row = [&](int q) -> int { return kPair ? (32 * (int)crank + 8 * pw) : (32 * q + 8 * pw); };
-    Cursor ca{m0.x, m0.y, 0}, cb = ca, cf = ca;   // rounds R+2 (stage A), R+1 (stage B), R (fill)
-    int64_t jf = 0;                                // tile index of round R
+    Cursor ca{m0.x, m0.y}, cb = ca, cf = ca;   // tiles t+2 (stage A), t+1 (stage B), t (fill)
 
-    int idx_a = -1, sl_a = 0;    // round R+2 (lanes 0-7)
-    int idx_b = -1, sl_b = 0;    // round R+1
-    int row_c = -1;              // round R: cache row of lane 0-7's slot, -1 if invalid
-    uint4 lat[8], rp[2];
-    float sc[8];
+    int idx_a = -1, sl_a = 0;    // tile t+2 (lanes 0..kRPW-1)
+    int idx_b = -1, sl_b = 0;    // tile t+1
+    int row_c = -1;              // tile t: cache row of lane k's slot, -1 if invalid
+    uint4 lat[kRPW], rp[kRPW / 4];
+    float sc[kRPW];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < kRPW; ++k) {
       lat[k] = make_uint4(0u, 0u, 0u, 0u);
       sc[k] = 0.f;
     }
-    rp[0] = rp[1] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int i = 0; i < kRPW / 4; ++i) rp[i] = make_uint4(0u, 0u, 0u, 0u);
 
     int req_ord = -1;
     bool ok = true;
 #pragma unroll 1
-    for (int64_t R = -2; R < nround && ok; ++R) {
-      // ---- stage A: index and request length of round R+2 -----------------
-      if (R + 2 < nround) {
-        const int slot = ca.t * kRows + first_row(ca.q) + lane;
+    for (int64_t R = -2; R < ntile && ok; ++R) {
+      // ---- stage A: index and request length of tile R+2 ------------------
+      if (R + 2 < ntile) {
+        const int slot = ca.t * kRows + rb + lane;
         idx_a = -1;
         sl_a = 0;
-        ldg_s32_if(idx_a, p.indices + (size_t)ca.r * p.topk + slot, lane < 8 && slot < p.topk);
-        ldg_s32_if(sl_a, p.seqlens + ca.r / p.s_q, lane < 8);
-        ca.advance(n, kRounds);
+        ldg_s32_if(idx_a, p.indices + (size_t)ca.r * p.topk + slot, lane < kRPW && slot < p.topk);
+        ldg_s32_if(sl_a, p.seqlens + ca.r / p.s_q, lane < kRPW);
+        ca.advance(n);
       }
-      // ---- stage B: block-table entry of round R+1 -------------------------
+      // ---- stage B: block-table entry of tile R+1 -------------------------
       int phys_b = -1;
-      if (R + 1 >= 0 && R + 1 < nround) {
-        const bool valid = lane < 8 && idx_b >= 0 && idx_b < sl_b;
+      if (R + 1 >= 0 && R + 1 < ntile) {
+        const bool valid = lane < kRPW && idx_b >= 0 && idx_b < sl_b;
         const int blk = idx_b >> 6;
         if (valid && blk >= p.max_blocks) report_status(p.status, kStatusBadBlockTable);
         ldg_s32_if(phys_b, p.block_table + (size_t)(cb.r / p.s_q) * p.max_blocks + blk,
                    valid && blk < p.max_blocks);
-        cb.advance(n, kRounds);
+        cb.advance(n);
       }
-      // ---- dequantise and store round R ------------------------------------
+      // ---- dequantise and store tile R -------------------------------------
       if (R >= 0) {
-        const int64_t j = jf;
-        const int q = cf.q;
+        const int64_t j = R;
         const bool tile_first = (j == 0) || (cf.t == 0);
         const int s = (int)(j & 1);
         const uint32_t aK = aK0 + (uint32_t)s * kTileBytes;
         const uint32_t aKr = kPair ? mapa_shared(aK, peer) : 0u;      // the peer's copy of this slot
-        if (q == 0) {
-          if (tile_first) {
-            ++req_ord;
-            if (req_ord > 0 &&
-                !mbar_wait_bounded_warp(&tail->qfree, (uint32_t)((req_ord - 1) & 1), kWaitLimitNs, p.status)) {
-              ok = false;
-              break;
-            }
-            const __nv_bfloat16* qsrc = p.q + ((size_t)cf.r * p.h_q + (size_t)kHeads * hg) * 576;
-#pragma unroll 1
-            for (int i0 = ptid; i0 < kHeads * 72; i0 += 128 * 6) {
-              uint4 v[6];
-#pragma unroll
-              for (int u = 0; u < 6; ++u) {
-                const int i = i0 + 128 * u;
-                const bool live = i < kHeads * 72 && i / 72 < heads_here;
-                v[u] = make_uint4(0u, 0u, 0u, 0u);
-                ldg_v4_if(v[u], qsrc + (live ? (size_t)(i / 72) * 576 + (i % 72) * 8 : 0), live);
-              }
-#pragma unroll
-              for (int u = 0; u < 6; ++u) {
-                const int i = i0 + 128 * u;
-                if (i < kHeads * 72) st_shared_v4(aQ + ((i % 72) >> 3) * kAtom + swz(i / 72, (i % 72) & 7), v[u]);
-              }
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&tail->qfull);
-          }
-          // the ring slot is free once PV of tile j-2 finished in every CTA of the cluster
-          if (!mbar_wait_bounded_warp(&tail->kempty[s], (uint32_t)(((j >> 1) & 1) ^ 1), kWaitLimitNs, p.status)) {
+        if (tile_first) {
+          ++req_ord;
+          if (req_ord > 0 &&
+              !mbar_wait_bounded_warp(&tail->qfree, (uint32_t)((req_ord - 1) & 1), kWaitLimitNs, p.status)) {
             ok = false;
             break;
           }
-        }
-        const int rb = first_row(q);
-        const uint32_t vbits = __ballot_sync(0xffffffffu, row_c >= 0) & 0xFFu;
+          const __nv_bfloat16* qsrc = p.q + ((size_t)cf.r * p.h_q + (size_t)kHeads * hg) * 576;
+          constexpr int kQThreads = 32 * kProducerWarps;
+#pragma unroll 1
+          for (int i0 = ptid; i0 < kHeads * 72; i0 += kQThreads * 3) {
+            uint4 v[3];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+            for (int u = 0; u < 3; ++u) {
+              const int i = i0 + kQThreads * u;
+              const bool live = i < kHeads * 72 && i / 72 < heads_here;
+              v[u] = make_uint4(0u, 0u, 0u, 0u);
+              ldg_v4_if(v[u], qsrc + (live ? (size_t)(i / 72) * 576 + (i % 72) * 8 : 0), live);
+            }
+#pragma unroll
+            for (int u = 0; u < 3; ++u) {
+              const int i = i0 + kQThreads * u;
+              if (i < kHeads * 72) st_shared_v4(aQ + ((i % 72) >> 3) * kAtom + swz(i / 72, (i % 72) & 7), v[u]);
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&tail->qfull);
+        }
+        // the ring slot is free once PV of tile j-2 finished in every CTA of the cluster
+        if (!mbar_wait_bounded_warp(&tail->kempty[s], (uint32_t)(((j >> 1) & 1) ^ 1), kWaitLimitNs, p.status)) {
+          ok = false;
+          break;
+        }
+        const uint32_t vbits = __ballot_sync(0xffffffffu, row_c >= 0) & ((1u << kRPW) - 1u);
+#pragma unroll
+        for (int k = 0; k < kRPW; ++k) {
           const int row = rb + k;
           uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
           if ((vbits >> k) & 1u) dequant16(lat[k], sc[k], lo, hi);
           const uint32_t o0 = kb * kAtom + swz(row, c_first);
           const uint32_t o1 = kb * kAtom + swz(row, c_second);
-          const uint4 v0 = swap ? hi : lo;
-          const uint4 v1 = swap ? lo : hi;
-          st_shared_v4(aK + o0, v0);
-          st_shared_v4(aK + o1, v1);
+          st_shared_v4(aK + o0, swap ? hi : lo);
+          st_shared_v4(aK + o1, swap ? lo : hi);
         }
 #pragma unroll
-        for (int i = 0; i < 2; ++i) st_shared_v4(aK + 8 * kAtom + swz(rb + 4 * i + (lane >> 3), lane & 7), rp[i]);
-        if (lane == 0) {
-          const uint32_t va = smem_u32(&tail->vmask[s][rb >> 3]);
-          st_shared_u8(va, vbits);
-          if (kPair) st_cluster_u8(mapa_shared(va, peer), vbits);
+        for (int i = 0; i < kRPW / 4; ++i) st_shared_v4(aK + 8 * kAtom + swz(rb + 4 * i + (lane >> 3), lane & 7), rp[i]);
+        // validity: one byte per 4-row group, bit k = row 4g+k
+        if (lane < kRPW / 4) {
+          const uint32_t va = smem_u32(&tail->vmask[s][(rb >> 2) + lane]);
+          const uint32_t nib = (vbits >> (4 * lane)) & 0xFu;
+          st_shared_u8(va, nib);
+          if (kPair) st_cluster_u8(mapa_shared(va, peer), nib);
         }
-        cf.advance(n, kRounds);
-        if (cf.q == 0) ++jf;
-        if (q == kRounds - 1) {
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tail->kfull[s]);
-          if (kPair) {
-            // The copy engine sends this warp's 8 rows (1 KB in each of the 9
-            // column blocks, same offsets) to the peer's slot; the peer's kfull
-            // counts the arrive and the 9 KB of completed copies.
-            const uint32_t rbar = mapa_shared(smem_u32(&tail->kfull[s]), peer);
-            if (lane == 0) mbar_arrive_expect_tx_cluster(rbar, kKBlocks * 8 * 128);
-            if (lane < kKBlocks) {
-              const uint32_t off = (uint32_t)(lane * kAtom + rb * 128);
-              bulk_copy_to_peer(aKr + off, aK + off, 8 * 128, rbar);
-            }
+        cf.advance(n);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tail->kfull[s]);
+        if (kPair) {
+          // The copy engine sends this warp's rows (kRPW x 128 bytes in each
+          // of the 9 column blocks, same offsets) to the peer's slot; the
+          // peer's kfull counts the arrive and the completed bytes.
+          const uint32_t rbar = mapa_shared(smem_u32(&tail->kfull[s]), peer);
+          if (lane == 0) mbar_arrive_expect_tx_cluster(rbar, kKBlocks * kRPW * 128);
+          if (lane < kKBlocks) {
+            const uint32_t off = (uint32_t)(lane * kAtom + rb * 128);
+            bulk_copy_to_peer(aKr + off, aK + off, kRPW * 128, rbar);
           }
         }
       }
-      // ---- stage C: row loads of round R+1 ---------------------------------
-      if (R + 1 >= 0 && R + 1 < nround) {
+      // ---- stage C: row loads of tile R+1 ----------------------------------
+      if (R + 1 >= 0 && R + 1 < ntile) {
         row_c = -1;
         if (phys_b >= p.num_blocks) report_status(p.status, kStatusBadBlockTable);
         else if (phys_b >= 0) row_c = phys_b * 64 + (idx_b & 63);
         // For every row, lane l takes latent bytes [16l, 16l+16) and the scale
-        // of its 128-value tile; the 8 x 8 RoPE chunks are spread two per
-        // lane (row l/8 and 4 + l/8, chunk l%8).
+        // of its 128-value tile; the RoPE chunks (8 per row) are spread over
+        // the lanes (row 4i + l/8, chunk l%8).
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < kRPW; ++k) {
           const int rk = __shfl_sync(0xffffffffu, row_c, k);
           const uint8_t* row = p.kv + (int64_t)max(rk, 0) * 656;
           lat[k] = make_uint4(0u, 0u, 0u, 0u);
@@ -392,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVP
           ldg_f32_evict_first_if(sc[k], row + 512 + 4 * (lane >> 3), rk >= 0, pol);
         }
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kRPW / 4; ++i) {
           const int rk = __shfl_sync(0xffffffffu, row_c, 4 * i + (lane >> 3));
           rp[i] = make_uint4(0u, 0u, 0u, 0u);
           ldg_v4_evict_first_if(rp[i], p.kv + (int64_t)max(rk, 0) * 656 + 528 + 16 * (lane & 7), rk >= 0, pol);
@@ -412,93 +473,81 @@ __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVP
     }
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer ====================================
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kHeads, kRows, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(kHeads, 256, true);
-      // Descriptors are built once; an MMA step only adds its byte offset >> 4
-      // to the start-address field (all addresses stay below 2^18).
-      const uint64_t dQ = smem_desc_sw128(aQ, 16, 1024);
-      const uint64_t dK0 = smem_desc_sw128(aK0, 16, 1024);
-      const uint64_t dP = smem_desc_sw128(aP, 16, 1024);
-      const uint64_t dV0 = smem_desc_sw128(aK0, kAtom, 1024);
-      int req_ord = -1;
-      int prev_req_ord = -1;
-      bool prev_first = false;
-      Cursor cm{m0.x, m0.y, 0};
-      // Iteration j issues S(j) and PV(j-1), whichever has its inputs first:
-      // the next scores are computed while the softmax warps turn S(j-1) into
-      // P(j-1), and a late tile j does not hold back PV(j-1) (whose commit
-      // frees a ring slot for the producers).  Readiness is polled with
-      // non-blocking tests; each barrier polled here cannot complete a second
-      // phase before the MMA this loop issues next.
+    // The whole warp runs this loop (so the descriptor arithmetic is
+    // warp-uniform); one elected lane issues each tcgen05 instruction.
+    const uint32_t idesc_s = idesc_bf16_f32(kHeads, kRows, false);
+    const uint32_t idesc_pv = idesc_bf16_f32(kHeads, 256, true);
+    // Descriptor lower halves (K-major operands: leading offset 16 bytes; V
+    // read MN-major: leading offset one column block) and the shared upper half.
+    const uint32_t q_lo = smem_desc_lo(aQ, 16);
+    const uint32_t k_lo0 = smem_desc_lo(aK0, 16);
+    const uint32_t p_lo = smem_desc_lo(aP, 16);
+    const uint32_t v_lo0 = smem_desc_lo(aK0, kAtom);
+    const uint32_t d_hi = smem_desc_hi_sw128(1024);
+    int req_ord = -1;
+    int prev_req_ord = -1;
+    bool prev_first = false;
+    Cursor cm{m0.x, m0.y};
+    // Iteration j issues S(j) and PV(j-1), whichever has its inputs first:
+    // the next scores are computed while the softmax warps turn S(j-1) into
+    // P(j-1), and a late tile j does not hold back PV(j-1) (whose commit
+    // frees a ring slot for the producers).  Readiness is polled with
+    // non-blocking tests; each barrier polled here cannot complete a second
+    // phase before the MMA this loop issues next.
 #pragma unroll 1
-      for (int64_t j = 0; j <= ntile; ++j) {
-        const bool t_first = (j == 0) || (cm.t == 0);
-        const bool t_last = (j == ntile - 1) || (cm.t == n - 1);
-        bool need_s = j < ntile, need_pv = j >= 1;
-        if (need_s && t_first) ++req_ord;
-        const int s = (int)(j & 1);
-        const int64_t i = j - 1;
-        const bool wait_drain = need_pv && prev_first && prev_req_ord > 0;
-        uint64_t t0 = 0;
-        bool stalled = false;
-        while (need_s || need_pv) {
-          bool went = false;
-          if (need_s && mbar_test_wait(&tail->kfull[s], (uint32_t)((j >> 1) & 1)) &&
-              (!t_first || mbar_test_wait(&tail->qfull, (uint32_t)(req_ord & 1)))) {
-            tc_fence_after();
-            const uint64_t dK = dK0 + (uint64_t)(((uint32_t)s * kTileBytes) >> 4);
-            const uint32_t d_s = tmem + kSCol + 64 * s;
-#pragma unroll 4
-            for (int kk = 0; kk < 36; ++kk) {
-              const uint64_t koff = (uint64_t)((((kk >> 2) * kAtom) + (kk & 3) * 32) >> 4);
-              mma_bf16_ss(d_s, dQ + koff, dK + koff, idesc_s, kk > 0);
-            }
-            if (t_last) mma_commit(&tail->qfree);
-            mma_commit(&tail->sfull[s]);
-            need_s = false;
-            went = true;
-          }
-          if (need_pv && mbar_test_wait(&tail->pfull, (uint32_t)(i & 1)) &&
-              (!wait_drain || mbar_test_wait(&tail->odrain, (uint32_t)((prev_req_ord - 1) & 1)))) {
-            tc_fence_after();
-            const uint64_t dV = dV0 + (uint64_t)(((uint32_t)(i & 1) * kTileBytes) >> 4);
-#pragma unroll 1
-            for (int ks = 0; ks < 4; ++ks) {
-#pragma unroll
-              for (int hh = 0; hh < 2; ++hh)
-                mma_bf16_ss(tmem + kOCol + ((uint32_t)(16 * hh) << 16), dP + (uint64_t)((ks * 32) >> 4),
-                            dV + (uint64_t)(((4 * hh) * kAtom + ks * 16 * 128) >> 4), idesc_pv,
-                            (ks > 0 || !prev_first) ? 1u : 0u);
-            }
-            if (kPair) mma_commit_multicast(&tail->kempty[i & 1], (uint16_t)0x3);
-            else mma_commit(&tail->kempty[i & 1]);
-            mma_commit(&tail->ofree);
-            need_pv = false;
-            went = true;
-          }
-          if (went) {
-            stalled = false;
-          } else if (!stalled) {
-            stalled = true;
-            t0 = global_timer_ns();
-          } else if (global_timer_ns() - t0 > kWaitLimitNs) {
-            report_status(p.status, kStatusTimeout);
-            break;
-          } else {
-            __nanosleep(kPollSleepNs);
-          }
+    for (int64_t j = 0; j <= ntile; ++j) {
+      const bool t_first = (j == 0) || (cm.t == 0);
+      const bool t_last = (j == ntile - 1) || (cm.t == n - 1);
+      bool need_s = j < ntile, need_pv = j >= 1;
+      if (need_s && t_first) ++req_ord;
+      const int s = (int)(j & 1);
+      const int64_t i = j - 1;
+      const bool wait_drain = need_pv && prev_first && prev_req_ord > 0;
+      uint64_t t0 = 0;
+      bool stalled = false;
+      while (need_s || need_pv) {
+        bool went = false;
+        if (need_s && mbar_test_wait_warp(&tail->kfull[s], (uint32_t)((j >> 1) & 1)) &&
+            (!t_first || mbar_test_wait_warp(&tail->qfull, (uint32_t)(req_ord & 1)))) {
+          tc_fence_after();
+          issue_s_tile(tmem + kSCol + 64 * s, q_lo, k_lo0 + (uint32_t)s * (kTileBytes >> 4), d_hi, idesc_s);
+          if (t_last) mma_commit(&tail->qfree);
+          mma_commit(&tail->sfull[s]);
+          need_s = false;
+          went = true;
         }
-        if (need_s || need_pv) break;
-        if (j < ntile) {
-          prev_first = t_first;
-          prev_req_ord = req_ord;
-          cm.advance(n, 1);
+        if (need_pv && mbar_test_wait_warp(&tail->pfull, (uint32_t)(i & 1)) &&
+            (!wait_drain || mbar_test_wait_warp(&tail->odrain, (uint32_t)((prev_req_ord - 1) & 1)))) {
+          tc_fence_after();
+          issue_pv_tile(tmem + kOCol, tmem + kOCol + (16u << 16), p_lo, v_lo0 + (uint32_t)(i & 1) * (kTileBytes >> 4),
+                        d_hi, idesc_pv, prev_first ? 0u : 1u);
+          if (kPair) mma_commit_multicast(&tail->kempty[i & 1], (uint16_t)0x3);
+          else mma_commit(&tail->kempty[i & 1]);
+          mma_commit(&tail->ofree);
+          need_pv = false;
+          went = true;
+        }
+        if (went) {
+          stalled = false;
+        } else if (!stalled) {
+          stalled = true;
+          t0 = global_timer_ns();
+        } else if (__shfl_sync(0xffffffffu, (global_timer_ns() - t0 > kWaitLimitNs) ? 1u : 0u, 0) != 0) {
+          if (lane == 0) report_status(p.status, kStatusTimeout);
+          break;
+        } else {
+          __nanosleep(kPollSleepNs);
         }
       }
-      // the last request's qfree arrive lands before the CTA may exit
-      if (ntile > 0) (void)mbar_wait_bounded(&tail->qfree, (uint32_t)(req_ord & 1), kWaitLimitNs, p.status);
+      if (need_s || need_pv) break;
+      if (j < ntile) {
+        prev_first = t_first;
+        prev_req_ord = req_ord;
+        cm.advance(n);
+      }
     }
+    // the last request's qfree arrive lands before the CTA may exit
+    if (ntile > 0) (void)mbar_wait_bounded_warp(&tail->qfree, (uint32_t)(req_ord & 1), kWaitLimitNs, p.status);
   } else {
     // ======================= softmax / epilogue (warps 0-3) =================
     // S is read from TMEM in two 32-column halves, twice: once for the row
@@ -510,9 +559,9 @@ __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVP
     int req_ord = -1;
     int slot = 0, nsplit = 1;
     bool req_ok = true;
-    Cursor cx{m0.x, m0.y, 0};
+    Cursor cx{m0.x, m0.y};
 #pragma unroll 1
-    for (int64_t j = 0; j < ntile; ++j, cx.advance(n, 1)) {
+    for (int64_t j = 0; j < ntile; ++j, cx.advance(n)) {
       struct {
         int r;
         bool first, last;
@@ -532,7 +581,9 @@ __global__ void __launch_bounds__(kThreads, 1) splitkv_mla_kernel(const SplitKVP
       if (!mbar_wait_bounded_warp(&tail->sfull[s], ph, kWaitLimitNs, p.status)) break;
       if (!mbar_wait_bounded_warp(&tail->kfull[s], ph, kWaitLimitNs, p.status)) break;
       tc_fence_after();
-      const uint64_t vm = ld_shared_u64(smem_u32(&tail->vmask[s][0]));
+      // 64 validity bits of this tile (the producers write one nibble per 4 rows)
+      const uint64_t vm = (uint64_t)nibbles_to_bits(ld_shared_u64(smem_u32(&tail->vmask[s][0]))) |
+                          ((uint64_t)nibbles_to_bits(ld_shared_u64(smem_u32(&tail->vmask[s][8]))) << 32);
       const uint32_t t_s = tmem + t_lane + kSCol + 64 * s;
       float mt = -INFINITY;
 #pragma unroll 1
