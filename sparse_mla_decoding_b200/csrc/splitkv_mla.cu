@@ -303,12 +303,14 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     // ======================= producers =====================================
     // Warp pw owns kRPW consecutive rows of every tile: 8 in the single-CTA
     // form, 4 in the two-CTA form (where a CTA dequantises 32 of the 64 rows
-    // and sends them to its peer).  Tiles are software-pipelined: the index
-    // of tile t+2 and the block-table entry of tile t+1 are loaded before
-    // tile t is dequantised, and the rows of tile t+1 right after it, so
-    // they are in flight while the warp waits for the next ring slot.  The
-    // loop body is kept small (one copy of each stage): the roles share the
-    // SM's instruction caches.
+    // and sends them to its peer).  Tiles are software-pipelined over four
+    // stages per iteration, in this order: dequantise tile t, load the rows
+    // of tile t+1, the block-table entries of tile t+2 and the indices of
+    // tile t+3.  Each stage reads what the next one loaded an iteration
+    // earlier, before that register is reloaded, so no load is waited on
+    // early, and the rows of tile t+1 are in flight while the warp waits for
+    // the next ring slot.  The loop body is kept small (one copy of each
+    // stage): the roles share the SM's instruction caches.
     constexpr int kRPW = kPair ? 4 : 8;
     const int pw = warp - 4;
     const int ptid = tid - 128;
@@ -321,11 +323,11 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     const int swap = (lane >> 2) & 1;
     const int c_first = 2 * (lane & 3) + swap;
     const int c_second = 2 * (lane & 3) + 1 - swap;
-    Cursor ca{m0.x, m0.y}, cb = ca, cf = ca;   // tiles t+2 (stage A), t+1 (stage B), t (fill)
+    Cursor ca{m0.x, m0.y}, cb = ca, cf = ca;   // tiles t+3 (indices), t+2 (block table), t (fill)
 
-    int idx_a = -1, sl_a = 0;    // tile t+2 (lanes 0..kRPW-1)
-    int idx_b = -1, sl_b = 0;    // tile t+1
-    int row_c = -1;              // tile t: cache row of lane k's slot, -1 if invalid
+    int idx = -1, sl = 0;        // index and request length of lane k's slot (lanes 0..kRPW-1)
+    int phys = -1, off = 0;      // its cache block (-1: skip) and row within the block
+    int row_c = -1;              // cache row of lane k's slot in the tile being dequantised
     uint4 lat[kRPW], rp[kRPW / 4];
     float sc[kRPW];
 #pragma unroll
@@ -339,26 +341,7 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     int req_ord = -1;
     bool ok = true;
 #pragma unroll 1
-    for (int64_t R = -2; R < ntile && ok; ++R) {
-      // ---- stage A: index and request length of tile R+2 ------------------
-      if (R + 2 < ntile) {
-        const int slot = ca.t * kRows + rb + lane;
-        idx_a = -1;
-        sl_a = 0;
-        ldg_s32_if(idx_a, p.indices + (size_t)ca.r * p.topk + slot, lane < kRPW && slot < p.topk);
-        ldg_s32_if(sl_a, p.seqlens + ca.r / p.s_q, lane < kRPW);
-        ca.advance(n);
-      }
-      // ---- stage B: block-table entry of tile R+1 -------------------------
-      int phys_b = -1;
-      if (R + 1 >= 0 && R + 1 < ntile) {
-        const bool valid = lane < kRPW && idx_b >= 0 && idx_b < sl_b;
-        const int blk = idx_b >> 6;
-        if (valid && blk >= p.max_blocks) report_status(p.status, kStatusBadBlockTable);
-        ldg_s32_if(phys_b, p.block_table + (size_t)(cb.r / p.s_q) * p.max_blocks + blk,
-                   valid && blk < p.max_blocks);
-        cb.advance(n);
-      }
+    for (int64_t R = -3; R < ntile && ok; ++R) {
       // ---- dequantise and store tile R -------------------------------------
       if (R >= 0) {
         const int64_t j = R;
@@ -435,11 +418,11 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
           }
         }
       }
-      // ---- stage C: row loads of tile R+1 ----------------------------------
+      // ---- row loads of tile R+1 -------------------------------------------
       if (R + 1 >= 0 && R + 1 < ntile) {
         row_c = -1;
-        if (phys_b >= p.num_blocks) report_status(p.status, kStatusBadBlockTable);
-        else if (phys_b >= 0) row_c = phys_b * 64 + (idx_b & 63);
+        if (phys >= p.num_blocks) report_status(p.status, kStatusBadBlockTable);
+        else if (phys >= 0) row_c = phys * 64 + off;
         // For every row, lane l takes latent bytes [16l, 16l+16) and the scale
         // of its 128-value tile; the RoPE chunks (8 per row) are spread over
         // the lanes (row 4i + l/8, chunk l%8).
@@ -459,8 +442,25 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
           ldg_v4_evict_first_if(rp[i], p.kv + (int64_t)max(rk, 0) * 656 + 528 + 16 * (lane & 7), rk >= 0, pol);
         }
       }
-      idx_b = idx_a;
-      sl_b = sl_a;
+      // ---- block-table entry of tile R+2 -----------------------------------
+      if (R + 2 >= 0 && R + 2 < ntile) {
+        const bool valid = lane < kRPW && idx >= 0 && idx < sl;
+        const int blk = idx >> 6;
+        if (valid && blk >= p.max_blocks) report_status(p.status, kStatusBadBlockTable);
+        off = idx & 63;
+        phys = -1;
+        ldg_s32_if(phys, p.block_table + (size_t)(cb.r / p.s_q) * p.max_blocks + blk, valid && blk < p.max_blocks);
+        cb.advance(n);
+      }
+      // ---- index and request length of tile R+3 ---------------------------
+      if (R + 3 < ntile) {
+        const int slot = ca.t * kRows + rb + lane;
+        idx = -1;
+        sl = 0;
+        ldg_s32_if(idx, p.indices + (size_t)ca.r * p.topk + slot, lane < kRPW && slot < p.topk);
+        ldg_s32_if(sl, p.seqlens + ca.r / p.s_q, lane < kRPW);
+        ca.advance(n);
+      }
     }
     // Every arrive aimed at this CTA's ring barriers (the peer's multicast
     // commits included) has landed before the CTA may exit: wait for the last
@@ -488,10 +488,11 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     int prev_req_ord = -1;
     bool prev_first = false;
     Cursor cm{m0.x, m0.y};
-    // Iteration j issues S(j) and PV(j-1), whichever has its inputs first:
-    // the next scores are computed while the softmax warps turn S(j-1) into
-    // P(j-1), and a late tile j does not hold back PV(j-1) (whose commit
-    // frees a ring slot for the producers).  Readiness is polled with
+    // Iteration j issues S(j) and PV(j-1), whichever has its inputs first
+    // (PV first when both are ready: its commit frees a ring slot for the
+    // producers and the O accumulator for the softmax warps).  The next
+    // scores are computed while the softmax warps turn S(j-1) into P(j-1),
+    // and a late tile j does not hold back PV(j-1).  Readiness is polled with
     // non-blocking tests; each barrier polled here cannot complete a second
     // phase before the MMA this loop issues next.
 #pragma unroll 1
@@ -507,15 +508,6 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       bool stalled = false;
       while (need_s || need_pv) {
         bool went = false;
-        if (need_s && mbar_test_wait_warp(&tail->kfull[s], (uint32_t)((j >> 1) & 1)) &&
-            (!t_first || mbar_test_wait_warp(&tail->qfull, (uint32_t)(req_ord & 1)))) {
-          tc_fence_after();
-          issue_s_tile(tmem + kSCol + 64 * s, q_lo, k_lo0 + (uint32_t)s * (kTileBytes >> 4), d_hi, idesc_s);
-          if (t_last) mma_commit(&tail->qfree);
-          mma_commit(&tail->sfull[s]);
-          need_s = false;
-          went = true;
-        }
         if (need_pv && mbar_test_wait_warp(&tail->pfull, (uint32_t)(i & 1)) &&
             (!wait_drain || mbar_test_wait_warp(&tail->odrain, (uint32_t)((prev_req_ord - 1) & 1)))) {
           tc_fence_after();
@@ -525,6 +517,15 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
           else mma_commit(&tail->kempty[i & 1]);
           mma_commit(&tail->ofree);
           need_pv = false;
+          went = true;
+        }
+        if (need_s && mbar_test_wait_warp(&tail->kfull[s], (uint32_t)((j >> 1) & 1)) &&
+            (!t_first || mbar_test_wait_warp(&tail->qfull, (uint32_t)(req_ord & 1)))) {
+          tc_fence_after();
+          issue_s_tile(tmem + kSCol + 64 * s, q_lo, k_lo0 + (uint32_t)s * (kTileBytes >> 4), d_hi, idesc_s);
+          if (t_last) mma_commit(&tail->qfree);
+          mma_commit(&tail->sfull[s]);
+          need_s = false;
           went = true;
         }
         if (went) {
@@ -550,12 +551,18 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     if (ntile > 0) (void)mbar_wait_bounded_warp(&tail->qfree, (uint32_t)(req_ord & 1), kWaitLimitNs, p.status);
   } else {
     // ======================= softmax / epilogue (warps 0-3) =================
-    // S is read from TMEM in two 32-column halves, twice: once for the row
-    // max, once for P (keeping the code and the register footprint small).
+    // Thread i of softmax warp w owns score row (head) 16 w + i % 16, columns
+    // [32 (i / 16), 32 (i / 16) + 32) of each tile (the 16x32bx2 TMEM shape);
+    // the two threads of a row combine their max and sum with one shuffle.
+    // P is computed before waiting for the previous PV, which only gates the
+    // P stores and the O rescale.  TMEM lane i of the O accumulator holds the
+    // same head (its upper lanes hold the second 256 columns), so the
+    // rescale factor is already in the right thread.
     const int my_head = 16 * warp + (lane & 15);
+    const int half = lane >> 4;
     const uint32_t t_lane = (uint32_t)(32 * warp) << 16;
     const float scale_log2 = p.scale_log2;
-    float m_used = -INFINITY, l_run = 0.f;
+    float m_used = -INFINITY, l_half = 0.f;
     int req_ord = -1;
     int slot = 0, nsplit = 1;
     bool req_ok = true;
@@ -571,7 +578,7 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       if (tp.first) {
         ++req_ord;
         m_used = -INFINITY;
-        l_run = 0.f;
+        l_half = 0.f;
         const int ns_r = p.num_splits[tp.r], ns_r1 = p.num_splits[tp.r + 1];
         slot = (req_ord == 0) ? m1.x : ns_r;
         nsplit = ns_r1 - ns_r;
@@ -581,34 +588,39 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       if (!mbar_wait_bounded_warp(&tail->sfull[s], ph, kWaitLimitNs, p.status)) break;
       if (!mbar_wait_bounded_warp(&tail->kfull[s], ph, kWaitLimitNs, p.status)) break;
       tc_fence_after();
-      // 64 validity bits of this tile (the producers write one nibble per 4 rows)
-      const uint64_t vm = (uint64_t)nibbles_to_bits(ld_shared_u64(smem_u32(&tail->vmask[s][0]))) |
-                          ((uint64_t)nibbles_to_bits(ld_shared_u64(smem_u32(&tail->vmask[s][8]))) << 32);
-      const uint32_t t_s = tmem + t_lane + kSCol + 64 * s;
+      // validity bits of this thread's 32 columns (one nibble per 4 rows)
+      const uint32_t vh = nibbles_to_bits(ld_shared_u64(smem_u32(&tail->vmask[s][8 * half])));
+      uint32_t sr[32];
+      tmem_ld16x2_32(tmem + t_lane + kSCol + 64 * s, sr);
+      tmem_wait_ld();
       float mt = -INFINITY;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        uint32_t sr[32];
-        tmem_ld32(t_s + 32 * h, sr);
-        tmem_wait_ld();
-        const uint32_t vh = (uint32_t)(vm >> (32 * h));
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if ((vh >> c) & 1u) mt = fmaxf(mt, __uint_as_float(sr[c]));
-      }
+      for (int c = 0; c < 32; ++c)
+        if ((vh >> c) & 1u) mt = fmaxf(mt, __uint_as_float(sr[c]));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
       float alpha = 1.f;
-      if (lane < 16) {
-        mt = (mt == -INFINITY) ? -INFINITY : mt * scale_log2;
-        if (mt > m_used + kRescaleLog2) {
-          alpha = fast_exp2(m_used - mt);     // 0 when nothing was valid before
-          l_run *= alpha;
-          m_used = mt;
-        }
+      mt = (mt == -INFINITY) ? -INFINITY : mt * scale_log2;
+      if (mt > m_used + kRescaleLog2) {
+        alpha = fast_exp2(m_used - mt);     // 0 when nothing was valid before
+        l_half *= alpha;
+        m_used = mt;
       }
+      // P = 2^(s * scale_log2 - m) for valid slots (0 otherwise), rounded to bf16
+      const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
+      float psum = 0.f;
+      uint32_t pk[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float p0 = ((vh >> (2 * c)) & 1u) ? fast_exp2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, neg_m)) : 0.f;
+        const float p1 =
+            ((vh >> (2 * c + 1)) & 1u) ? fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, neg_m)) : 0.f;
+        psum += p0 + p1;
+        pk[c] = bf162_bits(__floats2bfloat162_rn(p0, p1));
+      }
+      if (m_used != -INFINITY) l_half += psum;
       // PV of the previous tile must be done before P is overwritten or O rescaled.
       if (j >= 1 && !mbar_wait_bounded_warp(&tail->ofree, (uint32_t)((j - 1) & 1), kWaitLimitNs, p.status)) break;
       tc_fence_after();
-      alpha = __shfl_sync(0xffffffffu, alpha, lane & 15);
       if (!tp.first && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
@@ -621,31 +633,9 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         }
         tmem_wait_st();
       }
-      // P = 2^(s * scale_log2 - m) for valid slots (0 otherwise), rounded to bf16
-      const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-      float psum = 0.f;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        uint32_t sr[32];
-        tmem_ld32(t_s + 32 * h, sr);
-        tmem_wait_ld();
-        const uint32_t vh = (uint32_t)(vm >> (32 * h));
-        uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float p0 = ((vh >> (2 * c)) & 1u) ? fast_exp2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, neg_m)) : 0.f;
-          const float p1 =
-              ((vh >> (2 * c + 1)) & 1u) ? fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, neg_m)) : 0.f;
-          psum += p0 + p1;
-          pk[c] = bf162_bits(__floats2bfloat162_rn(p0, p1));
-        }
-        if (lane < 16) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            st_shared_v4(aP + swz(my_head, 4 * h + c), make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
-        }
-      }
-      if (m_used != -INFINITY) l_run += psum;
+      for (int c = 0; c < 4; ++c)
+        st_shared_v4(aP + swz(my_head, 4 * half + c), make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&tail->pfull);
@@ -653,9 +643,8 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       if (tp.last) {
         if (!mbar_wait_bounded_warp(&tail->ofree, (uint32_t)(j & 1), kWaitLimitNs, p.status)) break;
         tc_fence_after();
-        const float l_me = __shfl_sync(0xffffffffu, l_run, lane & 15);
-        const float m_me = __shfl_sync(0xffffffffu, m_used, lane & 15);
-        const int half = lane >> 4;
+        const float l_me = l_half + __shfl_xor_sync(0xffffffffu, l_half, 16);
+        const float m_me = m_used;
         const int head = kHeads * hg + my_head;
         const bool live = req_ok && (my_head < heads_here);
         const float inv_l = (l_me > 0.f) ? 1.f / l_me : 0.f;
