@@ -224,6 +224,28 @@ def make_device_copy(w, device):
                 indices=torch.from_numpy(idx).to(device), idx_host=idx, seqlens_host=lay.seqlens)
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one split-kernel
+# launch from an ncu capture, per workload, with the hash of the kernel sources
+# the capture was taken on (build.source_hash()).  Reported only while the
+# sources still match; the capture commands are in profiles/.
+NCU_TRAFFIC = {
+    "decode_h128_b64_topk2048": {
+        "bytes": 107_493_376 + 4_281_344,
+        "srchash": "4332c0164a04923f8d84a47d0d4609d11fa4d1cc5c4e9fad572d6883ebc46242"},
+    "decode_h64_b128_sq2_topk2048": {
+        "bytes": 395_659_264 + 4_271_616,
+        "srchash": "4332c0164a04923f8d84a47d0d4609d11fa4d1cc5c4e9fad572d6883ebc46242"},
+}
+
+
+def measured_traffic(workload):
+    from sparse_mla_decoding_b200 import build as B
+    rec = NCU_TRAFFIC.get(workload)
+    if rec is None or rec["srchash"] != B.source_hash():
+        return None
+    return rec["bytes"]
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -366,7 +388,7 @@ def run_ours(args, w, rank, world, local_rank):
         achieved = per_launch_bytes / (kern_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
-    roof.update({"traffic": None, "kernel": "splitkv_mla_kernel + combine_kernel (one decode call)",
+    roof.update({"traffic": measured_traffic(w.name), "kernel": "splitkv_mla_kernel + combine_kernel (one decode call)",
                  "kernel_ms": kern_ms, "peak_source": peaks["source"] + " (burst)"})
 
     line = {
