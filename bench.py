@@ -246,6 +246,26 @@ def measured_traffic(workload):
     return rec["bytes"]
 
 
+def rank_seed(w, rank, copy):
+    """Seed of input copy `copy` on rank `rank`: every rank and copy draws its own inputs."""
+    return w.seed + 1000 * rank + 17 * copy
+
+
+def reduce_over_ranks(times, work, device, world):
+    """Whole-job numbers: the max of each time and the sum of each work count over ranks.
+
+    Every rank calls it with the same list lengths, in the same order (NCCL on GPUs;
+    the CPU tests run it over gloo)."""
+    import torch
+    t = torch.tensor([float(x) for x in times], dtype=torch.float64, device=device)
+    s = torch.tensor([float(x) for x in work], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(s, op=dist.ReduceOp.SUM)
+    return t.tolist(), s.tolist()
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -258,10 +278,7 @@ def run_ours(args, w, rank, world, local_rank):
     stream = torch.cuda.current_stream(device)
 
     # independent copies (weak scaling: every rank has its own seeds)
-    copies = []
-    for c in range(args.copies):
-        wc = w.with_(seed=w.seed + 1000 * rank + 17 * c)
-        copies.append(make_device_copy(wc, device))
+    copies = [make_device_copy(w.with_(seed=rank_seed(w, rank, c)), device) for c in range(args.copies)]
     torch.cuda.synchronize()
     flops_per_copy = [step_flops(w.h_q, valid_counts(c["idx_host"], c["seqlens_host"])) for c in copies]
     valid_per_copy = [float(valid_counts(c["idx_host"], c["seqlens_host"]).sum()) for c in copies]
@@ -361,14 +378,8 @@ def run_ours(args, w, rank, world, local_rank):
         raise RuntimeError(f"device status word set during the benchmark: {raw:#x}")
 
     # ---- reduce over ranks (max time, summed work) --------------------------
-    vals = torch.tensor([ms_total, e2e_ms, kern_ms, my_flops, my_valid], dtype=torch.float64, device=device)
-    if world > 1:
-        mx = vals.clone()
-        dist.all_reduce(mx[:3], op=dist.ReduceOp.MAX)
-        sm_ = vals.clone()
-        dist.all_reduce(sm_[3:], op=dist.ReduceOp.SUM)
-        vals = torch.cat([mx[:3], sm_[3:]])
-    ms_total, e2e_ms, kern_ms, tot_flops, tot_valid = vals.tolist()
+    (ms_total, e2e_ms, kern_ms), (tot_flops, tot_valid) = reduce_over_ranks(
+        [ms_total, e2e_ms, kern_ms], [my_flops, my_valid], device, world)
     if rank != 0:
         return
 

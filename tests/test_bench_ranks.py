@@ -1,0 +1,94 @@
+"""The multi-rank logic of bench.py on CPU: two gloo ranks, no GPU.
+
+bench.py runs one process per GPU; on more than one rank the whole-job time is
+the max over ranks and the work is summed, rank 0 alone prints, and every rank
+draws its own inputs.  These tests run that logic over gloo with world size 2.
+"""
+import contextlib
+import io
+import json
+import os
+import socket
+import sys
+import tempfile
+import types
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    import datetime
+
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        # rank r: times (r + 1, 10 - r, 0.5 r), work (r + 1, 100)
+        times, work = bench.reduce_over_ranks([rank + 1.0, 10.0 - rank, 0.5 * rank], [rank + 1, 100], "cpu", world)
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump({"times": times, "work": work}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reduce_over_ranks_gloo_world2():
+    import torch.multiprocessing as mp
+
+    world = 2
+    with tempfile.TemporaryDirectory() as d:
+        mp.spawn(_rank_main, args=(world, _free_port(), d), nprocs=world, join=True)
+        res = [json.load(open(os.path.join(d, f"rank{r}.json"))) for r in range(world)]
+    for r in res:   # every rank ends with the same whole-job numbers
+        assert r["times"] == [2.0, 10.0, 0.5]
+        assert r["work"] == [3.0, 200.0]
+
+
+def test_single_rank_reduction_is_identity():
+    import bench
+
+    times, work = bench.reduce_over_ranks([3.5, 1.0], [7, 8], "cpu", 1)
+    assert times == [3.5, 1.0] and work == [7.0, 8.0]
+
+
+def test_rank_seeds_are_distinct():
+    import bench
+    from sparse_mla_decoding_b200 import workloads as W
+
+    w = W.BY_NAME["decode_h128_b64_topk2048"]
+    seeds = {bench.rank_seed(w, r, c) for r in range(8) for c in range(4)}
+    assert len(seeds) == 32
+
+
+def test_reference_arm_prints_on_rank0_only():
+    import bench
+    from sparse_mla_decoding_b200 import workloads as W
+
+    w = W.BY_NAME["tiny_h16_b2_topk64"]
+    args = types.SimpleNamespace(steps=1, warmup=0, gpus=2)
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.run_reference(args, w, rank=1, world=2)
+    assert buf.getvalue() == ""
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.run_reference(args, w, rank=0, world=2)
+    lines = [l for l in buf.getvalue().splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
