@@ -25,27 +25,36 @@
 //     (each CTA dequantises half of the rows, and the copy engine sends them
 //     to the peer with bulk shared-to-shared copies);
 //     16/32 heads are zero-padded to 64 in a single CTA.
-//   * Warp roles (288 threads):
-//       warps 0-3  softmax: online softmax over S in TMEM, P to shared memory,
-//                  lazy O rescaling, epilogue (own TMEM lane quarters 0-3);
-//       warps 4-7  producers: index -> page map, 16-byte coalesced gathers of
-//                  the 656-byte rows (evict-first), exact dequantisation into
-//                  a double-buffered 64 x 576 bf16 K ring (128-byte swizzled,
-//                  K-major; the same tile read MN-major is V), Q loads;
-//       warp 8     MMA issuer: the warp runs the issue loop, one elected lane
-//                  issues each MMA and commit; the warp owns TMEM.
-//   * Order of the MMAs: S(t+1) and PV(t) are issued as their inputs become
-//     ready, so the tensor core computes the next scores while the softmax
-//     warps work on the current ones, and a late tile never delays the PV
-//     that frees a ring slot.
-//   * The producers run a three-stage software pipeline across tiles: the
-//     indices of tile t+2 and the block-table entries of tile t+1 are loaded
-//     while tile t is dequantised, and the rows of tile t+1 right after, so
-//     the dependent loads index -> block table -> row never stall a tile.
-//   * TMEM (512 columns): O = 64 x 512 fp32 in columns [0, 256), its two
-//     256-wide halves in the lower and upper 16 lanes of each sub-partition
-//     (an M = 64 accumulator uses 16 lanes per sub-partition); S double
-//     buffer in columns [256, 320) and [320, 384), lanes 0-15.
+//   * Warp roles (416 threads, 13 warps, at most 128 registers a thread: one
+//     SM sub-partition holds 4 of the 13 warps):
+//       warps 0-3   softmax: online softmax over S in TMEM (two threads per
+//                   head row, 32 score columns each), P to shared memory,
+//                   lazy O rescaling, epilogue (own TMEM lane quarters 0-3);
+//       warps 4-11  producers: index -> page map, 16-byte coalesced gathers
+//                   of the 656-byte rows (evict-first), exact dequantisation
+//                   into a double-buffered 64 x 576 bf16 K ring (128-byte
+//                   swizzled, K-major; the same tile read MN-major is V), and
+//                   each request's Q into TMEM;
+//       warp 12     MMA issuer: the warp runs the issue loop, one elected
+//                   lane issues each MMA and commit; the warp owns TMEM.
+//   * MMAs: S = Q K^T with Q (the A operand) in TMEM and K in shared memory;
+//     PV = P V with P and V in shared memory.  S(t+1) and PV(t) are issued
+//     as their inputs become ready (PV first when both are), so the tensor
+//     core computes the next scores while the softmax warps work on the
+//     current ones, and a late tile never delays the PV that frees a ring
+//     slot.
+//   * The producers run a four-stage software pipeline across tiles
+//     (dequantise tile t, row loads of t+1, block table of t+2, indices of
+//     t+3), so the dependent loads index -> block table -> row never stall
+//     a tile and the rows are in flight while the ring slot drains.
+//   * TMEM (512 columns; an M = 64 operand or accumulator uses 16 lanes of
+//     each 32-lane sub-partition): lanes 0-15 hold Q (64 x 576 bf16, two
+//     values a column, columns [0, 288)) and the S double buffer (columns
+//     [320, 384) and [384, 448)); lanes 16-31 hold O = 64 x 512 fp32 in
+//     columns [0, 256) and [256, 512).
+//   * Shared memory: the K ring (2 x 72 KB) and P (8 KB), about 153 KB.
+//     Keeping Q out of it leaves the SM more L1 for the row gathers in
+//     flight and halves the shared-memory reads of the S MMAs.
 //   * Online softmax in base 2.  The running max used for P only moves when a
 //     tile's max exceeds it by more than 2^8 (then O and l are rescaled), so
 //     P <= 256 and rescales are rare; lse = (m + log2 l) ln 2 at the end.
@@ -77,10 +86,17 @@ constexpr int kAtom = kRows * 128;     // bytes of one 64-row x 128-byte column 
 constexpr int kTileBytes = kKBlocks * kAtom;
 constexpr int kPBytes = kAtom;
 static_assert(kAtom == 8192 && kKBlocks == 9, "the MMA blocks below encode 64-row column blocks as literal offsets");
-static_assert(3 * kTileBytes + kAtom < (1 << 18), "descriptor start fields are 14 bits of (address >> 4)");
+static_assert(2 * kTileBytes + kAtom < (1 << 18), "descriptor start fields are 14 bits of (address >> 4)");
+// TMEM (512 columns x 128 lanes; an M = 64 operand or accumulator uses 16
+// lanes of each 32-lane sub-partition):
+//   lanes 0-15 of each quarter: Q (64 x 576 bf16, two values per column) in
+//     columns [kQCol, kQCol + 288), S double buffer at kSCol + 64 s;
+//   lanes 16-31: O (64 x 512 fp32), columns [0, 256) and [256, 512).
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kOCol = 0;
-constexpr uint32_t kSCol = 256;        // S buffer s at kSCol + 64 s
+constexpr uint32_t kQCol = 0;
+constexpr uint32_t kSCol = 320;        // S buffer s at kSCol + 64 s, lanes 0-15
+constexpr uint32_t kOLane = 16;        // O in lanes 16-31
+static_assert(kQCol + 288 <= kSCol && kSCol + 128 <= kTmemCols, "TMEM column map");
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no legitimate wait comes close
 #ifndef SMLA_POLL_SLEEP_NS
@@ -102,9 +118,8 @@ struct __align__(16) Tail {
   uint8_t vmask[2][16];  // per K buffer: bit k of byte g = row 4g+k holds a valid slot
 };
 
-constexpr int kOffQ = 0;
-constexpr int kOffK = kTileBytes;
-constexpr int kOffP = 3 * kTileBytes;
+constexpr int kOffK = 0;
+constexpr int kOffP = 2 * kTileBytes;
 constexpr int kOffTail = kOffP + kPBytes;
 constexpr int kSmemBytes = kOffTail + (int)sizeof(Tail) + 1024;
 
@@ -115,30 +130,30 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk16) {
 __device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
 // One S tile: 36 MMAs (9 column blocks x 4 K-steps of 16) of M = 64, N = 64,
-// issued by one elected lane of a converged warp.  Operands: D column, Q and
-// K descriptor lower halves, the shared upper half, the instruction
-// descriptor.  A K-step adds 32 bytes (2 in descriptor units) and a column
-// block kAtom = 8192 bytes (512).
+// issued by one elected lane of a converged warp.  A = Q in TMEM (a K-step
+// is 8 columns, a column block 32); B = the K tile in shared memory (a K-step
+// adds 32 bytes = 2 descriptor units, a column block kAtom = 8192 bytes =
+// 512).  Operands: D column, Q TMEM address, K descriptor lower half, the
+// shared upper half, the instruction descriptor.
 #define SMLA_S_STEP(kb, k4, acc)                                       \
-  "add.u32 la, %1, (" #kb "*512+" #k4 "*2);\n\t"                       \
+  "add.u32 la, %1, (" #kb "*32+" #k4 "*8);\n\t"                        \
   "add.u32 lb, %2, (" #kb "*512+" #k4 "*2);\n\t"                       \
-  "mov.b64 da, {la, %3};\n\t"                                          \
   "mov.b64 db, {lb, %3};\n\t"                                          \
-  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, " acc ";\n\t"
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [la], db, %4, " acc ";\n\t"
 #define SMLA_S_BLOCK(kb) \
   SMLA_S_STEP(kb, 0, "pt") SMLA_S_STEP(kb, 1, "pt") SMLA_S_STEP(kb, 2, "pt") SMLA_S_STEP(kb, 3, "pt")
 
-__device__ __forceinline__ void issue_s_tile(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo, uint32_t hi,
+__device__ __forceinline__ void issue_s_tile(uint32_t d_tmem, uint32_t q_tmem, uint32_t k_lo, uint32_t hi,
                                              uint32_t idesc) {
   asm volatile(
-      "{\n\t.reg .pred e, pt, pf;\n\t.reg .b32 la, lb;\n\t.reg .b64 da, db;\n\t"
+      "{\n\t.reg .pred e, pt, pf;\n\t.reg .b32 la, lb;\n\t.reg .b64 db;\n\t"
       "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 pt, 1, 0;\n\t"
       "setp.eq.b32 pf, 1, 0;\n\t"
       SMLA_S_STEP(0, 0, "pf") SMLA_S_STEP(0, 1, "pt") SMLA_S_STEP(0, 2, "pt") SMLA_S_STEP(0, 3, "pt")
       SMLA_S_BLOCK(1) SMLA_S_BLOCK(2) SMLA_S_BLOCK(3) SMLA_S_BLOCK(4)
       SMLA_S_BLOCK(5) SMLA_S_BLOCK(6) SMLA_S_BLOCK(7) SMLA_S_BLOCK(8)
-      "}" ::"r"(d_tmem), "r"(q_lo), "r"(k_lo), "r"(hi), "r"(idesc)
+      "}" ::"r"(d_tmem), "r"(q_tmem), "r"(k_lo), "r"(hi), "r"(idesc)
       : "memory");
 }
 
@@ -241,7 +256,6 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Tail* tail = reinterpret_cast<Tail*>(smem + kOffTail);
-  const uint32_t aQ = smem_u32(smem + kOffQ);
   const uint32_t aK0 = smem_u32(smem + kOffK);
   const uint32_t aP = smem_u32(smem + kOffP);
 
@@ -356,25 +370,33 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
             ok = false;
             break;
           }
-          const __nv_bfloat16* qsrc = p.q + ((size_t)cf.r * p.h_q + (size_t)kHeads * hg) * 576;
-          constexpr int kQThreads = 32 * kProducerWarps;
+          // Q of this request into TMEM (lanes 0-15 of this warp's quarter):
+          // thread i holds head 16 (warp % 4) + i % 16 and, per 32-column chunk
+          // c, the 32 values [64 c + 32 (i / 16), +32) packed two to a column.
+          // The two producer warps of a quarter take chunks 0-4 and 5-8.
+          {
+            const int qh = 16 * (warp & 3) + (lane & 15);
+            const bool qlive = qh < heads_here;
+            const __nv_bfloat16* qrow = p.q + ((size_t)cf.r * p.h_q + (size_t)kHeads * hg + (qlive ? qh : 0)) * 576;
+            const uint32_t qaddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + kQCol;
+            const int c0 = (pw < 4) ? 0 : 5, c1 = (pw < 4) ? 5 : 9;
 #pragma unroll 1
-          for (int i0 = ptid; i0 < kHeads * 72; i0 += kQThreads * 3) {
-            uint4 v[3];
+            for (int c = c0; c < c1; ++c) {
+              uint32_t v[16];
 #pragma unroll
-            for (int u = 0; u < 3; ++u) {
-              const int i = i0 + kQThreads * u;
-              const bool live = i < kHeads * 72 && i / 72 < heads_here;
-              v[u] = make_uint4(0u, 0u, 0u, 0u);
-              ldg_v4_if(v[u], qsrc + (live ? (size_t)(i / 72) * 576 + (i % 72) * 8 : 0), live);
-            }
-#pragma unroll
-            for (int u = 0; u < 3; ++u) {
-              const int i = i0 + kQThreads * u;
-              if (i < kHeads * 72) st_shared_v4(aQ + ((i % 72) >> 3) * kAtom + swz(i / 72, (i % 72) & 7), v[u]);
+              for (int u = 0; u < 4; ++u) {
+                uint4 x = make_uint4(0u, 0u, 0u, 0u);
+                ldg_v4_if(x, qrow + 64 * c + 32 * (lane >> 4) + 8 * u, qlive);
+                v[4 * u] = x.x;
+                v[4 * u + 1] = x.y;
+                v[4 * u + 2] = x.z;
+                v[4 * u + 3] = x.w;
+              }
+              tmem_st16x2_16(qaddr + 32 * c, v);
             }
           }
-          fence_proxy_async_smem();
+          tmem_wait_st();
+          tc_fence_before();
           mbar_arrive(&tail->qfull);
         }
         // the ring slot is free once PV of tile j-2 finished in every CTA of the cluster
@@ -479,7 +501,6 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     const uint32_t idesc_pv = idesc_bf16_f32(kHeads, 256, true);
     // Descriptor lower halves (K-major operands: leading offset 16 bytes; V
     // read MN-major: leading offset one column block) and the shared upper half.
-    const uint32_t q_lo = smem_desc_lo(aQ, 16);
     const uint32_t k_lo0 = smem_desc_lo(aK0, 16);
     const uint32_t p_lo = smem_desc_lo(aP, 16);
     const uint32_t v_lo0 = smem_desc_lo(aK0, kAtom);
@@ -511,8 +532,8 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         if (need_pv && mbar_test_wait_warp(&tail->pfull, (uint32_t)(i & 1)) &&
             (!wait_drain || mbar_test_wait_warp(&tail->odrain, (uint32_t)((prev_req_ord - 1) & 1)))) {
           tc_fence_after();
-          issue_pv_tile(tmem + kOCol, tmem + kOCol + (16u << 16), p_lo, v_lo0 + (uint32_t)(i & 1) * (kTileBytes >> 4),
-                        d_hi, idesc_pv, prev_first ? 0u : 1u);
+          issue_pv_tile(tmem + (kOLane << 16), tmem + (kOLane << 16) + 256, p_lo,
+                        v_lo0 + (uint32_t)(i & 1) * (kTileBytes >> 4), d_hi, idesc_pv, prev_first ? 0u : 1u);
           if (kPair) mma_commit_multicast(&tail->kempty[i & 1], (uint16_t)0x3);
           else mma_commit(&tail->kempty[i & 1]);
           mma_commit(&tail->ofree);
@@ -522,7 +543,7 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         if (need_s && mbar_test_wait_warp(&tail->kfull[s], (uint32_t)((j >> 1) & 1)) &&
             (!t_first || mbar_test_wait_warp(&tail->qfull, (uint32_t)(req_ord & 1)))) {
           tc_fence_after();
-          issue_s_tile(tmem + kSCol + 64 * s, q_lo, k_lo0 + (uint32_t)s * (kTileBytes >> 4), d_hi, idesc_s);
+          issue_s_tile(tmem + kSCol + 64 * s, tmem + kQCol, k_lo0 + (uint32_t)s * (kTileBytes >> 4), d_hi, idesc_s);
           if (t_last) mma_commit(&tail->qfree);
           mma_commit(&tail->sfull[s]);
           need_s = false;
@@ -625,11 +646,11 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + t_lane + kOCol + 32 * c, o);
+          tmem_ld16x2_32(tmem + t_lane + (kOLane << 16) + 64 * c, o);
           tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          tmem_st32(tmem + t_lane + kOCol + 32 * c, o);
+          tmem_st16x2_32(tmem + t_lane + (kOLane << 16) + 64 * c, o);
         }
         tmem_wait_st();
       }
@@ -653,9 +674,9 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         for (int c = 0; c < 8; ++c) {
           uint32_t o[32];
           __syncwarp();
-          tmem_ld32(tmem + t_lane + kOCol + 32 * c, o);
+          tmem_ld16x2_32(tmem + t_lane + (kOLane << 16) + 64 * c, o);
           tmem_wait_ld();
-          const int col = half * 256 + 32 * c;
+          const int col = 64 * c + 32 * half;
           if (!live) {
           } else if (nsplit == 1) {
             __nv_bfloat16* dst = p.o + ((size_t)tp.r * p.h_q + head) * 512 + col;
