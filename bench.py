@@ -23,6 +23,7 @@ gathered rows were not left in L2 by the previous steps.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import signal
@@ -79,29 +80,45 @@ def load_peaks():
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock and throttle-reason samples (every 20 ms) around a timed region.
+
+    `mark_start()` / `mark_end()` bracket the timed region; the summary keeps the
+    samples whose timestamps fall inside it, widened by `pad_ms` on each side (a
+    region of a few milliseconds is shorter than nvidia-smi's sampling period, and
+    the warm-up right before it runs the same work)."""
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, pad_ms: float = 50.0):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.pad_ms = pad_ms
+        self.t_start = None
+        self.t_end = None
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                                          "--format=csv,noheader,nounits", "-lms", "20", "-f", self.path],
                                          stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except OSError:
             self.proc = None
         return self
 
+    def mark_start(self):
+        self.t_start = datetime.datetime.now()
+
+    def mark_end(self):
+        self.t_end = datetime.datetime.now()
+
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(0.1)   # let the sample after the region land
             self.proc.send_signal(signal.SIGTERM)
             try:
                 self.proc.wait(timeout=5)
@@ -109,27 +126,45 @@ class ClockSampler:
                 self.proc.kill()
         return False
 
-    def summary(self):
-        if not self.path or not os.path.exists(self.path):
-            return None
+    @staticmethod
+    def parse(lines):
         rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-                except ValueError:
-                    continue
-        os.remove(self.path)
+        for line in lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+            except ValueError:
+                ts = None
+            try:
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+            except ValueError:
+                continue
+        return rows
+
+    def summarize(self, rows):
+        window = f"timed region +- {self.pad_ms:.0f} ms"
+        if self.t_start is not None and self.t_end is not None and rows and all(r[0] is not None for r in rows):
+            pad = datetime.timedelta(milliseconds=self.pad_ms)
+            rows = [r for r in rows if self.t_start - pad <= r[0] <= self.t_end + pad]
+        else:
+            window = "whole sampler run (timestamps unavailable)"
         if not rows:
             return None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
-        sm = [r[0] for r in rows]
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
-                "samples": len(rows)}
+        reasons = sorted({names[i] for _, _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        sm = [r[1] for r in rows]
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(r[2] for r in rows), "reasons": reasons,
+                "samples": len(rows), "window": window}
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        with open(self.path) as f:
+            rows = self.parse(f.readlines())
+        os.remove(self.path)
+        return self.summarize(rows)
 
 
 # ---------------------------------------------------------------------------
@@ -230,11 +265,11 @@ def make_device_copy(w, device):
 # sources still match; the capture commands are in profiles/.
 NCU_TRAFFIC = {
     "decode_h128_b64_topk2048": {
-        "bytes": 107_493_376 + 4_281_344,
-        "srchash": "4332c0164a04923f8d84a47d0d4609d11fa4d1cc5c4e9fad572d6883ebc46242"},
+        "bytes": 107_550_720 + 5_125_376,
+        "srchash": "f46fc65068e16aa2fcecd14c604cb1694c0ddedd5ffab1947a7b34121fec30d4"},
     "decode_h64_b128_sq2_topk2048": {
-        "bytes": 395_659_264 + 4_271_616,
-        "srchash": "4332c0164a04923f8d84a47d0d4609d11fa4d1cc5c4e9fad572d6883ebc46242"},
+        "bytes": 395_680_768 + 5_133_056,
+        "srchash": "f46fc65068e16aa2fcecd14c604cb1694c0ddedd5ffab1947a7b34121fec30d4"},
 }
 
 
@@ -307,11 +342,13 @@ def run_ours(args, w, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         barrier()
         torch.cuda.synchronize()
+        clk.mark_start()
         ev0.record(stream)
         for i in range(args.steps):
             step(i % args.copies)
         ev1.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
         barrier()
     ms_total = ev0.elapsed_time(ev1)
     clocks = clk.summary()

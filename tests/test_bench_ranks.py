@@ -1,4 +1,5 @@
-"""The multi-rank logic of bench.py on CPU: two gloo ranks, no GPU.
+"""Host-side logic of bench.py on CPU, no GPU: the multi-rank path over two gloo ranks,
+the reference arm's rank gating and the clock sampler's window.
 
 bench.py runs one process per GPU; on more than one rank the whole-job time is
 the max over ranks and the work is summed, rank 0 alone prints, and every rank
@@ -92,3 +93,36 @@ def test_reference_arm_prints_on_rank0_only():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_clock_sampler_keeps_samples_of_the_timed_region():
+    import datetime
+
+    import bench
+
+    c = bench.ClockSampler(0, pad_ms=50.0)
+    lines = [
+        "2026/12/02 19:35:11.000, 0, 1000, 1965, 100.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/02 19:35:12.100, 0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/02 19:35:12.200, 0, 1900, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/02 19:35:13.900, 0, 210, 1965, 100.0, 0x0, Not Active, Active, Not Active, Not Active",
+        "garbage line",
+    ]
+    rows = c.parse(lines)
+    assert len(rows) == 4
+    c.t_start = datetime.datetime(2026, 12, 2, 19, 35, 12, 90000)
+    c.t_end = datetime.datetime(2026, 12, 2, 19, 35, 12, 160000)
+    s = c.summarize(rows)
+    assert s["samples"] == 2 and s["sm_mhz"] == 1932.5 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and "timed region" in s["window"]
+
+
+def test_clock_sampler_without_timestamps_uses_every_sample():
+    import bench
+
+    c = bench.ClockSampler(0)
+    rows = c.parse(["n/a, 0, 1800, 1965, 500.0, 0x0, Not Active, Not Active, Not Active, Not Active"])
+    c.mark_start()
+    c.mark_end()
+    s = c.summarize(rows)
+    assert s["samples"] == 1 and s["sm_mhz"] == 1800.0 and "whole sampler run" in s["window"]
