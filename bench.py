@@ -260,23 +260,34 @@ def make_device_copy(w, device):
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one split-kernel
-# launch from an ncu capture, per workload, with the hash of the kernel sources
-# the capture was taken on (build.source_hash()).  Reported only while the
-# sources still match; the capture commands are in profiles/.
+# launch from an ncu capture, per workload, with the hash of the split kernel's
+# sources and build flags the capture was taken on (split_kernel_hash()).
+# Reported only while they still match; the capture commands are in profiles/.
 NCU_TRAFFIC = {
     "decode_h128_b64_topk2048": {
         "bytes": 107_550_720 + 5_125_376,
-        "srchash": "f46fc65068e16aa2fcecd14c604cb1694c0ddedd5ffab1947a7b34121fec30d4"},
+        "srchash": "dc378b35c53c2791723f2adcf6c66e4763ab184b230c13c99d0fd6b47e36a918"},
     "decode_h64_b128_sq2_topk2048": {
         "bytes": 395_680_768 + 5_133_056,
-        "srchash": "f46fc65068e16aa2fcecd14c604cb1694c0ddedd5ffab1947a7b34121fec30d4"},
+        "srchash": "dc378b35c53c2791723f2adcf6c66e4763ab184b230c13c99d0fd6b47e36a918"},
 }
 
 
+def split_kernel_hash():
+    """Hash of the files the split kernel is compiled from (and of the build flags)."""
+    import hashlib
+    pkg = os.path.join(os.path.dirname(os.path.abspath(__file__)), "sparse_mla_decoding_b200")
+    h = hashlib.sha256()
+    for rel in ("csrc/splitkv_mla.cu", "csrc/sm100.cuh", "csrc/splitkv_mla.h", "build.py"):
+        h.update(rel.encode())
+        with open(os.path.join(pkg, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def measured_traffic(workload):
-    from sparse_mla_decoding_b200 import build as B
     rec = NCU_TRAFFIC.get(workload)
-    if rec is None or rec["srchash"] != B.source_hash():
+    if rec is None or rec["srchash"] != split_kernel_hash():
         return None
     return rec["bytes"]
 

@@ -145,6 +145,42 @@ int smla_flash_mla_with_kvcache(const void* q, const uint8_t* kvcache, int64_t n
                                 void* o, float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Sparse attention of many query tokens over one flat (unpaged) FP8 cache
+ * ("deepseek-ai/FlashMLA" (agentlenshq), section 使用方法 item 2:
+ * flash_mla_sparse_fwd(q, kv, indices, ...) with a 3-D indices tensor that
+ * names the KV tokens each query token attends to; 技術的な詳細: -1 marks a
+ * skipped entry).  Query token t and head h attend to the rows
+ * kv[indices[t][0][j]] with 0 <= indices[t][0][j] < s_kv, with the row
+ * format, dequantisation, scores, o and lse of smla_flash_mla_with_kvcache.
+ * Runs the decode path on batch 1 with s_q query tokens: a small kernel
+ * writes an identity block table and the request length into the
+ * workspace, then the scheduler, the split kernel and the combine run on
+ * `stream`.
+ *   q        : device bf16 [s_q][h_q][576] (16-byte aligned)
+ *   kv       : device uint8 [s_kv][656] (16-byte aligned), one KV head;
+ *              1 <= s_kv <= 2147483584
+ *   indices  : device int32 [s_q][1][topk]; negative or >= s_kv = skip
+ *   num_sm_parts : scheduler parts (smla_default_num_sm_parts(h_q, device))
+ *   softmax_scale : <= 0 or NaN selects the default 1/sqrt(576)
+ *   o        : device bf16 [s_q][h_q][512], written
+ *   lse      : device float32 [s_q][h_q], natural log, written
+ *   workspace: device, >= smla_sparse_fwd_workspace_bytes(...) bytes,
+ *              256-byte aligned; its first 256 bytes are the status header
+ *              (zero it once; read it with smla_get_device_status)
+ */
+int smla_flash_mla_sparse_fwd(const void* q, const uint8_t* kv, int64_t s_kv, const int32_t* indices, int s_q,
+                              int h_q, int topk, int num_sm_parts, float softmax_scale, void* o, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace bytes of smla_flash_mla_sparse_fwd: the decode workspace for
+ * (batch 1, s_q, h_q, topk, num_sm_parts), the scheduler tables, the
+ * request length and a block table of ceil(s_kv / 64) entries.  Returns 0
+ * for invalid arguments.
+ */
+size_t smla_sparse_fwd_workspace_bytes(int s_q, int h_q, int64_t s_kv, int topk, int num_sm_parts);
+
+/*
  * Write tokens into the 656-byte FP8 cache rows ("FlashMLA 注意力内核源码走读…",
  * section 数据加载: the first 512 dimensions are quantised per 1x128 tile):
  * per tile, scale = amax / 448 in float32, byte = e4m3(x / scale) rounded to

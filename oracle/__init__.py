@@ -257,6 +257,34 @@ def sparse_decode(q_bits: np.ndarray, kvcache: np.ndarray, block_table: np.ndarr
         return dict(ex.map(one, tokens))
 
 
+def sparse_prefill(q_bits: np.ndarray, kv_rows: np.ndarray, indices: np.ndarray,
+                   softmax_scale: float = DEFAULT_SOFTMAX_SCALE, tokens=None):
+    """Sparse attention of s_q query tokens over one flat FP8 cache.
+
+    Follows "deepseek-ai/FlashMLA" (agentlenshq), section 使用方法 item 2
+    (flash_mla_sparse_fwd(q, kv, indices, ...) with 3-D indices naming, per
+    query token, the KV tokens it attends to) and 技術的な詳細 (-1 = ignored):
+    token t attends to the rows kv_rows[i] of its indices with 0 <= i < s_kv,
+    each row taken through the same dequantisation and attention as the
+    sparse decode.  A flat cache is a paged one whose block table is the
+    identity, so this calls ``sparse_decode_token`` with that table; the rows
+    that pad the cache to whole 64-row blocks are never read.
+
+    q_bits [s_q, h, 576] bf16 bits; kv_rows [s_kv, 656] uint8; indices
+    [s_q, 1, topk] or [s_q, topk] int32.  Returns dict t -> (o [h, 512], lse [h]).
+    """
+    s_kv = kv_rows.shape[0]
+    nb = (s_kv + BLOCK - 1) // BLOCK
+    cache = np.zeros((nb * BLOCK, ROW_BYTES), dtype=np.uint8)
+    cache[:s_kv] = kv_rows.reshape(s_kv, ROW_BYTES)
+    cache = cache.reshape(nb, BLOCK, ROW_BYTES)
+    table = np.arange(nb, dtype=np.int32)
+    idx = indices.reshape(indices.shape[0], -1)
+    if tokens is None:
+        tokens = range(idx.shape[0])
+    return {t: sparse_decode_token(q_bits[t], cache, table, s_kv, idx[t], softmax_scale) for t in tokens}
+
+
 # --------------------------------------------------------------------------
 # scheduler metadata
 # --------------------------------------------------------------------------

@@ -58,6 +58,10 @@ def lib() -> ctypes.CDLL:
             L.smla_flash_mla_with_kvcache.argtypes = [vp, vp, i64, vp, i32, vp, vp, vp, vp, i32, f32, i32, i32, i32,
                                                       i32, vp, vp, vp, sz, vp]
             L.smla_flash_mla_with_kvcache.restype = i32
+            L.smla_flash_mla_sparse_fwd.argtypes = [vp, vp, i64, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+            L.smla_flash_mla_sparse_fwd.restype = i32
+            L.smla_sparse_fwd_workspace_bytes.argtypes = [i32, i32, i64, i32, i32]
+            L.smla_sparse_fwd_workspace_bytes.restype = sz
             L.smla_quantize_kv.argtypes = [vp, vp, i64, vp, vp, i64, vp]
             L.smla_quantize_kv.restype = i32
             L.smla_get_device_status.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_uint32), vp]
@@ -197,6 +201,68 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
         _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _check(rc, "smla_flash_mla_with_kvcache")
     return o, lse
+
+
+def sparse_fwd_workspace_bytes(s_q: int, h_q: int, s_kv: int, topk: int, num_sm_parts: int) -> int:
+    n = lib().smla_sparse_fwd_workspace_bytes(s_q, h_q, s_kv, topk, num_sm_parts)
+    if n == 0:
+        raise SmlaError(1, "smla_sparse_fwd_workspace_bytes")
+    return int(n)
+
+
+def flash_mla_sparse_fwd(q: torch.Tensor, kv: torch.Tensor, indices: torch.Tensor,
+                         softmax_scale: Optional[float] = None, num_sm_parts: Optional[int] = None,
+                         workspace: Optional[torch.Tensor] = None,
+                         out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None
+                         ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Sparse attention of s_q query tokens over one flat FP8 cache: (o bf16 [s_q, h_q, 512], lse [s_q, h_q]).
+
+    q: bf16 [s_q, h_q, 576]; kv: uint8 [s_kv, (1,) 656] (656-byte rows, one KV head);
+    indices: int32 [s_q, 1, topk] (or [s_q, topk]), negative or >= s_kv = skip.
+    A workspace from new_sparse_fwd_workspace may be passed; its first 256 bytes are
+    the device status word (get_device_status).
+    """
+    _require(q.is_cuda and q.dtype == torch.bfloat16 and q.dim() == 3 and q.shape[-1] == D_QK,
+             "q must be a bf16 CUDA tensor [s_q, h_q, 576]")
+    s_q, h_q, _ = q.shape
+    _require(kv.dtype == torch.uint8 and kv.shape[-1] == KV_ROW_BYTES and kv.dim() in (2, 3) and
+             (kv.dim() == 2 or kv.shape[1] == 1), "kv must be uint8 [s_kv, (1,) 656]")
+    _require(indices.dtype == torch.int32 and indices.shape[0] == s_q and
+             (indices.dim() == 2 or (indices.dim() == 3 and indices.shape[1] == 1)),
+             "indices must be int32 [s_q, 1, topk] or [s_q, topk]")
+    for name, t in (("kv", kv), ("indices", indices)):
+        _require(t.is_cuda and t.device == q.device, f"{name} must be on {q.device}")
+        _require(t.is_contiguous(), f"{name} must be contiguous")
+    q = q.contiguous()
+    s_kv = kv.shape[0]
+    topk = indices.shape[-1]
+    dev = q.device
+    if num_sm_parts is None:
+        num_sm_parts = default_num_sm_parts(h_q, dev)
+    nbytes = sparse_fwd_workspace_bytes(s_q, h_q, s_kv, topk, num_sm_parts)
+    if workspace is None:
+        workspace = _cached_workspace(dev, nbytes)
+    _require(workspace.is_cuda and workspace.numel() * workspace.element_size() >= nbytes,
+             f"workspace needs {nbytes} bytes")
+    if out is None:
+        o = torch.empty((s_q, h_q, D_V), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((s_q, h_q), dtype=torch.float32, device=dev)
+    else:
+        o, lse = out
+    scale = -1.0 if softmax_scale is None else float(softmax_scale)
+    rc = lib().smla_flash_mla_sparse_fwd(_ptr(q), _ptr(kv), s_kv, _ptr(indices), s_q, h_q, topk, int(num_sm_parts),
+                                         scale, _ptr(o), _ptr(lse), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(dev))
+    _check(rc, "smla_flash_mla_sparse_fwd")
+    return o, lse
+
+
+def new_sparse_fwd_workspace(s_q: int, h_q: int, s_kv: int, topk: int, num_sm_parts: int,
+                             device: Optional[torch.device] = None) -> torch.Tensor:
+    """A zeroed workspace for flash_mla_sparse_fwd (the zeroed header is the device status word)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return torch.zeros(sparse_fwd_workspace_bytes(s_q, h_q, s_kv, topk, num_sm_parts), dtype=torch.uint8,
+                       device=dev)
 
 
 def quantize_kv(latent: torch.Tensor, rope: torch.Tensor, kvcache: torch.Tensor,

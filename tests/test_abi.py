@@ -89,6 +89,34 @@ def test_argument_checks_return_before_launch():
     assert L.smla_selftest_bounded_wait(None, 1000, None) == 1
 
 
+def test_sparse_fwd_workspace_and_argument_checks():
+    L = smla.lib()
+    fake = ctypes.c_void_p(0x10000)
+    # workspace = decode workspace (batch 1) + scheduler tables + length + block table, each 256-rounded
+    s_q, h_q, s_kv, topk, P = 130, 64, 1000, 200, 8
+    dec = L.smla_workspace_bytes(1, s_q, h_q, topk, P)
+    up = lambda x: (x + 255) // 256 * 256
+    nb = (s_kv + 63) // 64
+    expect = up(dec) + up(P * 8 * 4) + up((s_q + 1) * 4) + 256 + up(nb * 4)
+    assert L.smla_sparse_fwd_workspace_bytes(s_q, h_q, s_kv, topk, P) == expect
+    assert L.smla_sparse_fwd_workspace_bytes(s_q, 48, s_kv, topk, P) == 0
+    assert L.smla_sparse_fwd_workspace_bytes(s_q, h_q, 0, topk, P) == 0
+    assert L.smla_sparse_fwd_workspace_bytes(s_q, h_q, (2 ** 31 - 1) // 64 * 64 + 1, topk, P) == 0
+    args = [fake, fake, s_kv, fake, s_q, h_q, topk, P, -1.0, fake, fake, fake, 1 << 30, None]
+    bad = list(args); bad[5] = 96                                    # h_q
+    assert L.smla_flash_mla_sparse_fwd(*bad) == 2
+    bad = list(args); bad[0] = None                                  # q
+    assert L.smla_flash_mla_sparse_fwd(*bad) == 1
+    bad = list(args); bad[2] = 0                                     # s_kv
+    assert L.smla_flash_mla_sparse_fwd(*bad) == 1
+    bad = list(args); bad[11] = ctypes.c_void_p(0x10010)             # workspace not 256-aligned
+    assert L.smla_flash_mla_sparse_fwd(*bad) == 1
+    bad = list(args); bad[12] = expect - 1                           # workspace too small
+    assert L.smla_flash_mla_sparse_fwd(*bad) == 1
+    bad = list(args); bad[6] = 0                                     # topk
+    assert L.smla_flash_mla_sparse_fwd(*bad) == 1
+
+
 def test_python_binding_shape_checks():
     import torch
     with pytest.raises(ValueError):

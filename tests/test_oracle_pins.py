@@ -15,6 +15,8 @@ an invariant that the definition of the method fixes:
     closed forms for one valid slot and for n identical rows
   * paging: gathering through a permuted block table equals gathering from a
     logically ordered cache; poisoned rows past the length are never read
+  * sparse prefill (flat cache): textbook attention over the rows each query
+    token names, with out-of-range and negative indices skipped
   * scheduler: brute-force enumeration of the tile ranges
 """
 import math
@@ -358,6 +360,27 @@ def test_paged_validity_rules_and_poison():
     o_ref, lse_ref = _textbook(q, Kl[keep], 1.0 / 24.0)
     assert np.isfinite(o).all()
     assert _close(o, o_ref) and _close(lse, lse_ref)
+
+
+def test_sparse_prefill_equals_textbook_over_its_rows():
+    # flat cache of 150 rows (not a whole number of 64-row blocks), values on the e4m3 grid
+    rng = np.random.default_rng(33)
+    s_kv = 150
+    cache, Kl = _grid_cache(rng, s_kv, 3, np.arange(3))
+    kv_rows = cache.reshape(-1, 656)[:s_kv].copy()
+    s_q, h = 5, 16
+    q_bits = _bits(rng.standard_normal((s_q, h, DQK)))
+    idx = rng.integers(-3, s_kv + 8, size=(s_q, 1, 40)).astype(np.int32)
+    idx[2, 0, :] = -1                                    # a token with no valid slot
+    ref = oracle.sparse_prefill(q_bits, kv_rows, idx)
+    for t in range(s_q):
+        keep = [int(i) for i in idx[t, 0] if 0 <= i < s_kv]
+        o, lse = ref[t]
+        if not keep:
+            assert (o == 0).all() and np.isneginf(lse).all()
+            continue
+        o_ref, lse_ref = _textbook(oracle.bf16_bits_to_f64(q_bits[t]), Kl[keep], 1.0 / 24.0)
+        assert _close(o, o_ref) and _close(lse, lse_ref)
 
 
 def test_sparse_decode_batch_driver():
