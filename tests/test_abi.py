@@ -121,3 +121,12 @@ def test_python_binding_shape_checks():
     import torch
     with pytest.raises(ValueError):
         smla.get_mla_metadata(torch.zeros(3, dtype=torch.int32), 64, 16, 8)     # not on CUDA
+    q = torch.zeros((4, 16, 576), dtype=torch.bfloat16)
+    kv = torch.zeros((10, 656), dtype=torch.uint8)
+    idx = torch.zeros((4, 1, 8), dtype=torch.int32)
+    with pytest.raises(ValueError):
+        smla.flash_mla_sparse_fwd(q, kv, idx)                                  # not on CUDA
+    with pytest.raises(ValueError):
+        smla.flash_mla_with_kvcache(q[None], kv.view(1, 10, 656), idx.view(1, 4, 8), torch.zeros(1, dtype=torch.int32),
+                                    idx.view(1, 4, 8), torch.zeros((8, 8), dtype=torch.int32),
+                                    torch.zeros(5, dtype=torch.int32))           # not on CUDA
