@@ -76,6 +76,14 @@ const char* smla_status_string(int status);
 int smla_version(void);
 
 /*
+ * The CUDA runtime error (a cudaError_t value) behind the most recent
+ * SMLA_ERR_CUDA that this host thread received, and its name (a static
+ * string, never NULL).  0 / "cudaSuccess" before any such failure.
+ */
+int smla_last_cuda_error(void);
+const char* smla_last_cuda_error_string(void);
+
+/*
  * Default number of scheduler parts for h_q heads on `device`: one part per
  * CTA group that can be resident at once (the SM count for h_q <= 64; half of
  * it for h_q = 128, where a part is a pair of CTAs that own 64 heads each).

@@ -25,7 +25,10 @@ from . import build as _build
 
 D_QK, D_V, D_ROPE, KV_ROW_BYTES, BLOCK_SIZE, INDEX_TILE = 576, 512, 64, 656, 64, 64
 STATUS_NAMES = {0: "SMLA_OK", 1: "SMLA_ERR_INVALID_ARGUMENT", 2: "SMLA_ERR_UNSUPPORTED", 3: "SMLA_ERR_CUDA",
-                4: "SMLA_ERR_DEVICE_TIMEOUT"}
+                4: "SMLA_ERR_DEVICE_TIMEOUT", 5: "SMLA_ERR_SCRATCH_LIMIT"}
+# Raw flag bits of the device status word (kernel side, sticky until reset).
+STATUS_FLAGS = {1: "a bounded device wait gave up", 2: "a valid index mapped outside the block table or the cache",
+                4: "scheduler metadata inconsistent with the call's shapes"}
 
 _lib = None
 _lib_lock = threading.Lock()
@@ -49,6 +52,10 @@ def lib() -> ctypes.CDLL:
             L.smla_status_string.restype = ctypes.c_char_p
             L.smla_version.argtypes = []
             L.smla_version.restype = i32
+            L.smla_last_cuda_error.argtypes = []
+            L.smla_last_cuda_error.restype = i32
+            L.smla_last_cuda_error_string.argtypes = []
+            L.smla_last_cuda_error_string.restype = ctypes.c_char_p
             L.smla_default_num_sm_parts.argtypes = [i32, i32]
             L.smla_default_num_sm_parts.restype = i32
             L.smla_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
@@ -76,6 +83,8 @@ def lib() -> ctypes.CDLL:
 
 def _check(rc: int, what: str) -> None:
     if rc != 0:
+        if rc == 3:   # SMLA_ERR_CUDA: name the CUDA runtime error behind it
+            what = f"{what} ({lib().smla_last_cuda_error_string().decode()})"
         raise SmlaError(rc, what)
 
 
@@ -118,14 +127,60 @@ _ws_cache: dict = {}
 _ws_lock = threading.Lock()
 
 
+def _ws_key(device: torch.device):
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    idx = dev.index if dev.index is not None else torch.cuda.current_device()
+    return idx, torch.cuda.current_stream(idx).cuda_stream
+
+
 def _cached_workspace(device: torch.device, nbytes: int) -> torch.Tensor:
-    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    """The workspace used when a call passes none: one per (device, current stream).
+
+    When a call needs more room, the buffer is replaced by a larger one and the
+    old status header (the sticky device status word) is carried over on the
+    stream, so flags raised by earlier calls are not lost.
+    """
+    key = _ws_key(device)
     with _ws_lock:
         ws = _ws_cache.get(key)
         if ws is None or ws.numel() < nbytes:
-            ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+            new = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+            if ws is not None:
+                new[:256].copy_(ws[:256])
+            ws = new
             _ws_cache[key] = ws
     return ws
+
+
+def cached_workspace_status(device: Optional[torch.device] = None) -> Tuple[int, int]:
+    """(status, raw flags) of the device status word of the workspace that calls
+    without a `workspace` argument share on `device` and the current stream.
+
+    Kernels record skipped bad block-table entries, inconsistent scheduler
+    metadata and bounded waits that gave up there; the flags stay set until
+    reset_cached_workspace_status.  Synchronises the current stream.
+    (0, 0) if no such call has run yet.
+    """
+    with _ws_lock:
+        ws = _ws_cache.get(_ws_key(device))
+    if ws is None:
+        return 0, 0
+    return get_device_status(ws)
+
+
+def reset_cached_workspace_status(device: Optional[torch.device] = None) -> None:
+    """Clear the status word of the shared workspace on `device` and the current stream."""
+    with _ws_lock:
+        ws = _ws_cache.get(_ws_key(device))
+    if ws is not None:
+        reset_device_status(ws)
+
+
+def _raise_on_flags(workspace: torch.Tensor, what: str) -> None:
+    st, raw = get_device_status(workspace)
+    if st != 0:
+        why = "; ".join(v for k, v in STATUS_FLAGS.items() if raw & k) or f"flags {raw:#x}"
+        raise SmlaError(st, f"{what} (device status: {why})")
 
 
 def get_mla_metadata(cache_seqlens: torch.Tensor, topk: int, h_q: int, num_sm_parts: Optional[int] = None,
@@ -152,7 +207,8 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
                            cache_seqlens: torch.Tensor, indices: torch.Tensor, sched_meta: torch.Tensor,
                            num_splits: torch.Tensor, softmax_scale: Optional[float] = None,
                            workspace: Optional[torch.Tensor] = None,
-                           out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None
+                           out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                           check_device_status: bool = False
                            ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Sparse MLA decode: returns (o bf16 [b, s_q, h_q, 512], lse float32 [b, s_q, h_q]).
 
@@ -160,6 +216,12 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
     block_table: int32 [b, max_blocks]; cache_seqlens: int32 [b];
     indices: int32 [b, s_q, topk] (negative or >= seqlen = skip);
     sched_meta / num_splits from get_mla_metadata with the same shapes.
+    Device-side problems (a valid index whose block lies outside the block
+    table or the cache, inconsistent metadata, a wait that gave up) set flags
+    in the workspace's status word: read them with get_device_status(workspace),
+    or with cached_workspace_status() when no workspace was passed.
+    check_device_status=True synchronises after the call and raises SmlaError
+    if any flag is set.
     """
     _require(q.is_cuda and q.dtype == torch.bfloat16 and q.dim() == 4 and q.shape[-1] == D_QK,
              "q must be a bf16 CUDA tensor [b, s_q, h_q, 576]")
@@ -200,6 +262,8 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
         _ptr(indices), _ptr(sched_meta), _ptr(num_splits), num_sm_parts, scale, b, s_q, h_q, topk, _ptr(o),
         _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _check(rc, "smla_flash_mla_with_kvcache")
+    if check_device_status:
+        _raise_on_flags(workspace, "smla_flash_mla_with_kvcache")
     return o, lse
 
 
@@ -213,7 +277,8 @@ def sparse_fwd_workspace_bytes(s_q: int, h_q: int, s_kv: int, topk: int, num_sm_
 def flash_mla_sparse_fwd(q: torch.Tensor, kv: torch.Tensor, indices: torch.Tensor,
                          softmax_scale: Optional[float] = None, num_sm_parts: Optional[int] = None,
                          workspace: Optional[torch.Tensor] = None,
-                         out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None
+                         out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                         check_device_status: bool = False
                          ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Sparse attention of s_q query tokens over one flat FP8 cache: (o bf16 [s_q, h_q, 512], lse [s_q, h_q]).
 
@@ -254,6 +319,8 @@ def flash_mla_sparse_fwd(q: torch.Tensor, kv: torch.Tensor, indices: torch.Tenso
                                          scale, _ptr(o), _ptr(lse), _ptr(workspace),
                                          workspace.numel() * workspace.element_size(), _stream(dev))
     _check(rc, "smla_flash_mla_sparse_fwd")
+    if check_device_status:
+        _raise_on_flags(workspace, "smla_flash_mla_sparse_fwd")
     return o, lse
 
 

@@ -16,6 +16,7 @@
 #include <cstring>
 
 #include "../../include/smla.h"
+#include "splitkv_mla.h"
 
 namespace smla {
 
@@ -86,7 +87,7 @@ int smla_flash_mla_sparse_fwd(const void* q, const uint8_t* kv, int64_t s_kv, co
   const int threads = 256;
   const int blocks = (nb + threads - 1) / threads < 1024 ? (nb + threads - 1) / threads : 1024;
   smla::sparse_fwd_setup_kernel<<<blocks, threads, 0, st>>>(seqlen, table, nb, (int32_t)s_kv);
-  if (cudaGetLastError() != cudaSuccess) return SMLA_ERR_CUDA;
+  if (const cudaError_t e = cudaGetLastError(); e != cudaSuccess) return smla::cuda_failure(e);
   if (int rc = smla_get_mla_metadata(seqlen, 1, s_q, topk, h_q, num_sm_parts, sched_meta, num_splits, stream))
     return rc;
   return smla_flash_mla_with_kvcache(q, kv, nb, table, nb, seqlen, indices, sched_meta, num_splits, num_sm_parts,

@@ -35,14 +35,15 @@
 //                   into a double-buffered 64 x 576 bf16 K ring (128-byte
 //                   swizzled, K-major; the same tile read MN-major is V), and
 //                   each request's Q into TMEM;
-//       warp 12     MMA issuer: the warp runs the issue loop, one elected
-//                   lane issues each MMA and commit; the warp owns TMEM.
-//   * MMAs: S = Q K^T with Q (the A operand) in TMEM and K in shared memory;
-//     PV = P V with P and V in shared memory.  S(t+1) and PV(t) are issued
-//     as their inputs become ready (PV first when both are), so the tensor
+//       warp 12     S issuer: waits for each K tile and issues its score
+//                   MMAs (one elected lane issues each MMA and commit); the
+//                   warp owns TMEM.
+//   * MMAs: S = Q K^T with Q (the A operand) in TMEM and K in shared memory,
+//     issued by warp 12 as soon as a tile is in shared memory, so the tensor
 //     core computes the next scores while the softmax warps work on the
-//     current ones, and a late tile never delays the PV that frees a ring
-//     slot.
+//     current ones; PV = P V with P and V in shared memory, issued by the
+//     softmax warpgroup itself right after it has written P (no hand-off to
+//     another warp on the per-tile critical path).
 //   * The producers run a four-stage software pipeline across tiles
 //     (dequantise tile t, row loads of t+1, block table of t+2, indices of
 //     t+3), so the dependent loads index -> block table -> row never stall
@@ -52,7 +53,8 @@
 //     values a column, columns [0, 288)) and the S double buffer (columns
 //     [320, 384) and [384, 448)); lanes 16-31 hold O = 64 x 512 fp32 in
 //     columns [0, 256) and [256, 512).
-//   * Shared memory: the K ring (2 x 72 KB) and P (8 KB), about 153 KB.
+//   * Shared memory: the K ring (2 x 72 KB) and a double-buffered P
+//     (2 x 8 KB), about 161 KB.
 //     Keeping Q out of it leaves the SM more L1 for the row gathers in
 //     flight and halves the shared-memory reads of the S MMAs.
 //   * Online softmax in base 2.  The running max used for P only moves when a
@@ -62,6 +64,7 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include <cstddef>
 #include <cstdint>
 #include <cstring>
 
@@ -84,9 +87,9 @@ constexpr int kRegCapThreads = 512;
 constexpr int kKBlocks = 9;            // 576 / 64 bf16 per 128-byte swizzle line
 constexpr int kAtom = kRows * 128;     // bytes of one 64-row x 128-byte column block
 constexpr int kTileBytes = kKBlocks * kAtom;
-constexpr int kPBytes = kAtom;
+constexpr int kPBytes = 2 * kAtom;   // P double buffer
 static_assert(kAtom == 8192 && kKBlocks == 9, "the MMA blocks below encode 64-row column blocks as literal offsets");
-static_assert(2 * kTileBytes + kAtom < (1 << 18), "descriptor start fields are 14 bits of (address >> 4)");
+static_assert(2 * kTileBytes + kPBytes < (1 << 18), "descriptor start fields are 14 bits of (address >> 4)");
 // TMEM (512 columns x 128 lanes; an M = 64 operand or accumulator uses 16
 // lanes of each 32-lane sub-partition):
 //   lanes 0-15 of each quarter: Q (64 x 576 bf16, two values per column) in
@@ -99,24 +102,21 @@ constexpr uint32_t kOLane = 16;        // O in lanes 16-31
 static_assert(kQCol + 288 <= kSCol && kSCol + 128 <= kTmemCols, "TMEM column map");
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no legitimate wait comes close
-#ifndef SMLA_POLL_SLEEP_NS
-#define SMLA_POLL_SLEEP_NS 32
-#endif
-constexpr uint32_t kPollSleepNs = SMLA_POLL_SLEEP_NS;  // MMA issuer back-off between readiness polls
 
 struct __align__(16) Tail {
+  // per K buffer: bit k of byte g = row 4g+k holds a valid slot (read as
+  // 8-byte words, so it stays first in the 16-byte aligned struct)
+  uint8_t vmask[2][16];
   uint64_t kfull[2];   // K tile s written (producers of both CTAs of a pair)
   uint64_t kempty[2];  // K tile s consumed by PV (both CTAs of a pair)
   uint64_t sfull[2];   // S buffer s computed
-  uint64_t pfull;      // P written and O rescaled
   uint64_t ofree;      // PV complete
-  uint64_t odrain;     // epilogue read O
+  uint64_t pready;     // the four softmax warps stored P (phase j for tile j)
   uint64_t qfull;      // Q tile loaded
   uint64_t qfree;      // last S of a request complete: sQ reusable
   uint32_t tmem_base;
-  int32_t abort;
-  uint8_t vmask[2][16];  // per K buffer: bit k of byte g = row 4g+k holds a valid slot
 };
+static_assert(offsetof(Tail, vmask) % 16 == 0 && offsetof(Tail, kfull) % 8 == 0, "Tail field alignment");
 
 constexpr int kOffK = 0;
 constexpr int kOffP = 2 * kTileBytes;
@@ -249,6 +249,22 @@ struct Cursor {
   }
 };
 
+// The same walk that also tracks the batch entry b = r / s_q of the request
+// (b and q = r % s_q advance with r, so the loop needs no division).
+struct BatchCursor {
+  int r, t, b, q;
+  __device__ __forceinline__ void advance(int n, int s_q) {
+    if (++t == n) {
+      t = 0;
+      ++r;
+      if (++q == s_q) {
+        q = 0;
+        ++b;
+      }
+    }
+  }
+};
+
 }  // namespace
 
 template <bool kPair>
@@ -274,12 +290,10 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       mbar_init(&tail->kempty[s], kPair ? 2 : 1);
       mbar_init(&tail->sfull[s], 1);
     }
-    mbar_init(&tail->pfull, 128);
     mbar_init(&tail->ofree, 1);
-    mbar_init(&tail->odrain, 128);
+    mbar_init(&tail->pready, 4);
     mbar_init(&tail->qfull, 32 * kProducerWarps);
     mbar_init(&tail->qfree, 1);
-    tail->abort = 0;
     fence_mbarrier_init();
   }
   if (warp == kMmaWarp) {
@@ -327,7 +341,6 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     // stage): the roles share the SM's instruction caches.
     constexpr int kRPW = kPair ? 4 : 8;
     const int pw = warp - 4;
-    const int ptid = tid - 128;
     const uint64_t pol = l2_evict_first_policy();
     const int rb = kPair ? (32 * (int)crank + kRPW * pw) : kRPW * pw;   // this warp's first row of a tile
     // Stores: lane l writes the two 16-byte halves of its 32-byte output in
@@ -337,10 +350,13 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     const int swap = (lane >> 2) & 1;
     const int c_first = 2 * (lane & 3) + swap;
     const int c_second = 2 * (lane & 3) + 1 - swap;
-    Cursor ca{m0.x, m0.y}, cb = ca, cf = ca;   // tiles t+3 (indices), t+2 (block table), t (fill)
+    // tiles t+3 (indices), t+2 (block table), t (fill)
+    BatchCursor ca{m0.x, m0.y, m0.x / p.s_q, m0.x % p.s_q}, cb = ca;
+    Cursor cf{m0.x, m0.y};
 
     int idx = -1, sl = 0;        // index and request length of lane k's slot (lanes 0..kRPW-1)
     int phys = -1, off = 0;      // its cache block (-1: skip) and row within the block
+    bool looked_up = false;      // lane k's slot is valid and its block-table entry was read
     int row_c = -1;              // cache row of lane k's slot in the tile being dequantised
     uint4 lat[kRPW], rp[kRPW / 4];
     float sc[kRPW];
@@ -405,15 +421,18 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
           break;
         }
         const uint32_t vbits = __ballot_sync(0xffffffffu, row_c >= 0) & ((1u << kRPW) - 1u);
+        // A skipped slot's registers were zeroed and its loads predicated
+        // off, so dequantising it unconditionally stores a zero row.  Lanes
+        // that store their upper half first swap the two 8-byte halves of
+        // the input instead of the two 16-byte halves of the output.
 #pragma unroll
         for (int k = 0; k < kRPW; ++k) {
           const int row = rb + k;
-          uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-          if ((vbits >> k) & 1u) dequant16(lat[k], sc[k], lo, hi);
-          const uint32_t o0 = kb * kAtom + swz(row, c_first);
-          const uint32_t o1 = kb * kAtom + swz(row, c_second);
-          st_shared_v4(aK + o0, swap ? hi : lo);
-          st_shared_v4(aK + o1, swap ? lo : hi);
+          const uint4 in = swap ? make_uint4(lat[k].z, lat[k].w, lat[k].x, lat[k].y) : lat[k];
+          uint4 first, second;
+          dequant16(in, sc[k], first, second);
+          st_shared_v4(aK + kb * kAtom + swz(row, c_first), first);
+          st_shared_v4(aK + kb * kAtom + swz(row, c_second), second);
         }
 #pragma unroll
         for (int i = 0; i < kRPW / 4; ++i) st_shared_v4(aK + 8 * kAtom + swz(rb + 4 * i + (lane >> 3), lane & 7), rp[i]);
@@ -442,9 +461,11 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       }
       // ---- row loads of tile R+1 -------------------------------------------
       if (R + 1 >= 0 && R + 1 < ntile) {
+        // A valid slot whose block-table entry lies outside the cache
+        // (negative or past num_blocks) is skipped and flagged.
         row_c = -1;
-        if (phys >= p.num_blocks) report_status(p.status, kStatusBadBlockTable);
-        else if (phys >= 0) row_c = phys * 64 + off;
+        if (phys >= 0 && phys < p.num_blocks) row_c = phys * 64 + off;
+        else if (looked_up) report_status(p.status, kStatusBadBlockTable);
         // For every row, lane l takes latent bytes [16l, 16l+16) and the scale
         // of its 128-value tile; the RoPE chunks (8 per row) are spread over
         // the lanes (row 4i + l/8, chunk l%8).
@@ -471,8 +492,9 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         if (valid && blk >= p.max_blocks) report_status(p.status, kStatusBadBlockTable);
         off = idx & 63;
         phys = -1;
-        ldg_s32_if(phys, p.block_table + (size_t)(cb.r / p.s_q) * p.max_blocks + blk, valid && blk < p.max_blocks);
-        cb.advance(n);
+        looked_up = valid && blk < p.max_blocks;
+        ldg_s32_if(phys, p.block_table + (size_t)cb.b * p.max_blocks + blk, looked_up);
+        cb.advance(n, p.s_q);
       }
       // ---- index and request length of tile R+3 ---------------------------
       if (R + 3 < ntile) {
@@ -480,8 +502,8 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         idx = -1;
         sl = 0;
         ldg_s32_if(idx, p.indices + (size_t)ca.r * p.topk + slot, lane < kRPW && slot < p.topk);
-        ldg_s32_if(sl, p.seqlens + ca.r / p.s_q, lane < kRPW);
-        ca.advance(n);
+        ldg_s32_if(sl, p.seqlens + ca.b, lane < kRPW);
+        ca.advance(n, p.s_q);
       }
     }
     // Every arrive aimed at this CTA's ring barriers (the peer's multicast
@@ -494,79 +516,32 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       }
     }
   } else if (warp == kMmaWarp) {
-    // ======================= MMA issuer ====================================
+    // ======================= S issuer ======================================
     // The whole warp runs this loop (so the descriptor arithmetic is
-    // warp-uniform); one elected lane issues each tcgen05 instruction.
+    // warp-uniform); one elected lane issues each tcgen05 instruction.  S(j)
+    // goes to TMEM buffer j % 2 as soon as K tile j is in shared memory: the
+    // softmax warps read S(j - 2) from that buffer before they issued PV(j - 2),
+    // and the producers refilled the ring slot of tile j only after PV(j - 2)
+    // completed, so the buffer is free.
     const uint32_t idesc_s = idesc_bf16_f32(kHeads, kRows, false);
-    const uint32_t idesc_pv = idesc_bf16_f32(kHeads, 256, true);
-    // Descriptor lower halves (K-major operands: leading offset 16 bytes; V
-    // read MN-major: leading offset one column block) and the shared upper half.
-    const uint32_t k_lo0 = smem_desc_lo(aK0, 16);
-    const uint32_t p_lo = smem_desc_lo(aP, 16);
-    const uint32_t v_lo0 = smem_desc_lo(aK0, kAtom);
+    const uint32_t k_lo0 = smem_desc_lo(aK0, 16);     // K-major: leading offset 16 bytes
     const uint32_t d_hi = smem_desc_hi_sw128(1024);
     int req_ord = -1;
-    int prev_req_ord = -1;
-    bool prev_first = false;
     Cursor cm{m0.x, m0.y};
-    // Iteration j issues S(j) and PV(j-1), whichever has its inputs first
-    // (PV first when both are ready: its commit frees a ring slot for the
-    // producers and the O accumulator for the softmax warps).  The next
-    // scores are computed while the softmax warps turn S(j-1) into P(j-1),
-    // and a late tile j does not hold back PV(j-1).  Readiness is polled with
-    // non-blocking tests; each barrier polled here cannot complete a second
-    // phase before the MMA this loop issues next.
 #pragma unroll 1
-    for (int64_t j = 0; j <= ntile; ++j) {
+    for (int64_t j = 0; j < ntile; ++j, cm.advance(n)) {
       const bool t_first = (j == 0) || (cm.t == 0);
       const bool t_last = (j == ntile - 1) || (cm.t == n - 1);
-      bool need_s = j < ntile, need_pv = j >= 1;
-      if (need_s && t_first) ++req_ord;
       const int s = (int)(j & 1);
-      const int64_t i = j - 1;
-      const bool wait_drain = need_pv && prev_first && prev_req_ord > 0;
-      uint64_t t0 = 0;
-      bool stalled = false;
-      while (need_s || need_pv) {
-        bool went = false;
-        if (need_pv && mbar_test_wait_warp(&tail->pfull, (uint32_t)(i & 1)) &&
-            (!wait_drain || mbar_test_wait_warp(&tail->odrain, (uint32_t)((prev_req_ord - 1) & 1)))) {
-          tc_fence_after();
-          issue_pv_tile(tmem + (kOLane << 16), tmem + (kOLane << 16) + 256, p_lo,
-                        v_lo0 + (uint32_t)(i & 1) * (kTileBytes >> 4), d_hi, idesc_pv, prev_first ? 0u : 1u);
-          if (kPair) mma_commit_multicast(&tail->kempty[i & 1], (uint16_t)0x3);
-          else mma_commit(&tail->kempty[i & 1]);
-          mma_commit(&tail->ofree);
-          need_pv = false;
-          went = true;
-        }
-        if (need_s && mbar_test_wait_warp(&tail->kfull[s], (uint32_t)((j >> 1) & 1)) &&
-            (!t_first || mbar_test_wait_warp(&tail->qfull, (uint32_t)(req_ord & 1)))) {
-          tc_fence_after();
-          issue_s_tile(tmem + kSCol + 64 * s, tmem + kQCol, k_lo0 + (uint32_t)s * (kTileBytes >> 4), d_hi, idesc_s);
-          if (t_last) mma_commit(&tail->qfree);
-          mma_commit(&tail->sfull[s]);
-          need_s = false;
-          went = true;
-        }
-        if (went) {
-          stalled = false;
-        } else if (!stalled) {
-          stalled = true;
-          t0 = global_timer_ns();
-        } else if (__shfl_sync(0xffffffffu, (global_timer_ns() - t0 > kWaitLimitNs) ? 1u : 0u, 0) != 0) {
-          if (lane == 0) report_status(p.status, kStatusTimeout);
-          break;
-        } else {
-          __nanosleep(kPollSleepNs);
-        }
+      if (t_first) {
+        ++req_ord;
+        if (!mbar_wait_bounded_warp(&tail->qfull, (uint32_t)(req_ord & 1), kWaitLimitNs, p.status)) break;
       }
-      if (need_s || need_pv) break;
-      if (j < ntile) {
-        prev_first = t_first;
-        prev_req_ord = req_ord;
-        cm.advance(n);
-      }
+      if (!mbar_spin_bounded_warp(&tail->kfull[s], (uint32_t)((j >> 1) & 1), kWaitLimitNs, p.status)) break;
+      tc_fence_after();
+      issue_s_tile(tmem + kSCol + 64 * s, tmem + kQCol, k_lo0 + (uint32_t)s * (kTileBytes >> 4), d_hi, idesc_s);
+      if (t_last) mma_commit(&tail->qfree);
+      mma_commit(&tail->sfull[s]);
     }
     // the last request's qfree arrive lands before the CTA may exit
     if (ntile > 0) (void)mbar_wait_bounded_warp(&tail->qfree, (uint32_t)(req_ord & 1), kWaitLimitNs, p.status);
@@ -575,14 +550,23 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     // Thread i of softmax warp w owns score row (head) 16 w + i % 16, columns
     // [32 (i / 16), 32 (i / 16) + 32) of each tile (the 16x32bx2 TMEM shape);
     // the two threads of a row combine their max and sum with one shuffle.
-    // P is computed before waiting for the previous PV, which only gates the
-    // P stores and the O rescale.  TMEM lane i of the O accumulator holds the
-    // same head (its upper lanes hold the second 256 columns), so the
-    // rescale factor is already in the right thread.
+    // P(j) goes to shared-memory buffer j % 2, which PV(j - 2) read: that MMA
+    // completed before the producers refilled the ring slot S(j) was computed
+    // from, so only an O rescale waits for the previous PV.  Once the four
+    // warps have stored P (named barrier), warp 0 issues PV(j) and commits
+    // the ring slot and the O accumulator.  The rendezvous is an mbarrier
+    // that only warp 0 waits on, with the usual time bound, so a warp that
+    // gives up cannot leave the others blocked.  TMEM lane i of the O accumulator
+    // holds the same head (its upper lanes hold the second 256 columns), so
+    // the rescale factor is already in the right thread.
     const int my_head = 16 * warp + (lane & 15);
     const int half = lane >> 4;
     const uint32_t t_lane = (uint32_t)(32 * warp) << 16;
     const float scale_log2 = p.scale_log2;
+    const uint32_t idesc_pv = idesc_bf16_f32(kHeads, 256, true);
+    const uint32_t p_lo0 = smem_desc_lo(aP, 16);        // P K-major: leading offset 16 bytes
+    const uint32_t v_lo0 = smem_desc_lo(aK0, kAtom);    // V read MN-major: leading offset one column block
+    const uint32_t d_hi = smem_desc_hi_sw128(1024);
     float m_used = -INFINITY, l_half = 0.f;
     int req_ord = -1;
     int slot = 0, nsplit = 1;
@@ -639,10 +623,11 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         pk[c] = bf162_bits(__floats2bfloat162_rn(p0, p1));
       }
       if (m_used != -INFINITY) l_half += psum;
-      // PV of the previous tile must be done before P is overwritten or O rescaled.
-      if (j >= 1 && !mbar_wait_bounded_warp(&tail->ofree, (uint32_t)((j - 1) & 1), kWaitLimitNs, p.status)) break;
-      tc_fence_after();
+      // An O rescale needs PV(j - 1) complete (this warpgroup issues every PV,
+      // so the parity of ofree's current phase cannot run ahead of j - 1).
       if (!tp.first && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!mbar_wait_bounded_warp(&tail->ofree, (uint32_t)((j - 1) & 1), kWaitLimitNs, p.status)) break;
+        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           uint32_t o[32];
@@ -654,12 +639,23 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         }
         tmem_wait_st();
       }
+      const uint32_t aPs = aP + (uint32_t)s * kAtom;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        st_shared_v4(aP + swz(my_head, 4 * half + c), make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
+        st_shared_v4(aPs + swz(my_head, 4 * half + c), make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&tail->pfull);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->pready);
+      if (warp == 0) {
+        if (!mbar_spin_bounded_warp(&tail->pready, (uint32_t)(j & 1), kWaitLimitNs, p.status)) break;
+        tc_fence_after();
+        issue_pv_tile(tmem + (kOLane << 16), tmem + (kOLane << 16) + 256, p_lo0 + (uint32_t)s * (kAtom >> 4),
+                      v_lo0 + (uint32_t)s * (kTileBytes >> 4), d_hi, idesc_pv, tp.first ? 0u : 1u);
+        if (kPair) mma_commit_multicast(&tail->kempty[s], (uint16_t)0x3);
+        else mma_commit(&tail->kempty[s]);
+        mma_commit(&tail->ofree);
+      }
 
       if (tp.last) {
         if (!mbar_wait_bounded_warp(&tail->ofree, (uint32_t)(j & 1), kWaitLimitNs, p.status)) break;
@@ -706,8 +702,9 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
           if (nsplit == 1) p.lse[(size_t)tp.r * p.h_q + head] = lse_val;
           else p.lse_accum[(size_t)slot * p.h_q + head] = lse_val;
         }
+        // The next request's first PV (issued by warp 0 after the next named
+        // barrier) overwrites O only after every warp's reads above.
         tc_fence_before();
-        mbar_arrive(&tail->odrain);
       }
     }
   }

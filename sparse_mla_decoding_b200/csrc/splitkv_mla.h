@@ -1,9 +1,12 @@
-// splitkv_mla.h -- parameters of the split-KV sparse MLA decode kernel (device side).
+// splitkv_mla.h -- internal interface between the decode entry points and the
+// split-KV sparse MLA decode kernels (device parameters, launchers and the
+// host-side pieces every decode entry point shares).
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cstddef>
 #include <cstdint>
 
 namespace smla {
@@ -29,12 +32,71 @@ struct SplitKVParams {
   uint32_t* status;             // sticky status word
 };
 
-// Dynamic shared memory of the split kernel, its one-time attribute set-up
-// (per device) and its launch (single CTA for <= 64 heads, a two-CTA cluster
-// for 128 heads; chained to the previous kernel with programmatic dependent
-// launch).
+// Heads merged by one CTA of the combine kernel (one warp per head).
+constexpr int kCombineHeadsPerCta = 8;
+
+// Dynamic shared memory of the split kernel, its attribute set-up (for the
+// current device) and its launch (single CTA for <= 64 heads, a two-CTA
+// cluster for 128 heads; chained to the previous kernel with programmatic
+// dependent launch).
 int splitkv_smem_bytes();
 cudaError_t configure_splitkv();
 cudaError_t launch_splitkv(const SplitKVParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// Host side shared by smla_flash_mla_with_kvcache and its allocation-free
+// variant, so both size, check and launch the decode the same way.
+// ---------------------------------------------------------------------------
+
+// A decode call's arguments as the C ABI receives them.
+struct DecodeCall {
+  const void* q;
+  const uint8_t* kvcache;
+  int64_t num_blocks;
+  const int32_t* block_table;
+  int max_blocks;
+  const int32_t* cache_seqlens;
+  const int32_t* indices;
+  const int32_t* sched_meta;
+  const int32_t* num_splits;
+  int num_sm_parts;
+  float softmax_scale;
+  int batch, s_q, h_q, topk;
+  void* o;
+  float* lse;
+};
+
+// Records a failing CUDA runtime result for smla_last_cuda_error (one slot
+// per host thread) and returns SMLA_ERR_CUDA.
+int cuda_failure(cudaError_t e);
+int g_last_cuda_error_value();
+
+// Scratch layout of a decode: a 256-byte status header, then float32
+// o_accum [max_splits][h_q][512] and lse_accum [max_splits][h_q], each
+// starting 256-byte aligned, with max_splits = batch * s_q + num_sm_parts.
+constexpr size_t kStatusHeaderBytes = 256;
+struct WorkspaceLayout {
+  size_t o_accum_off, lse_accum_off, total;
+};
+WorkspaceLayout workspace_layout(int batch, int s_q, int h_q, int num_sm_parts);
+
+// Host-side checks of a decode call (everything but the scratch): an
+// smla_status code, SMLA_OK when the call may be launched.  A call with
+// batch == 0 passes and launches nothing.
+int check_decode_call(const DecodeCall& c);
+
+// The current CUDA context as an opaque handle (nullptr if it cannot be
+// queried).  Module-level state (kernel attributes, the device address of a
+// __device__ array) belongs to a context, which cudaDeviceReset replaces.
+void* current_context();
+
+// Makes the split kernel launchable on the current device (sm_100 check and
+// the dynamic shared-memory attribute), once per device and CUDA context.
+int ensure_decode_kernels();
+
+// Launches the split kernel and, chained to it, the combine kernel, with
+// the partials in `scratch` (laid out by workspace_layout) and the sticky
+// status word at `status`.  The call must have passed check_decode_call.
+int launch_decode(const DecodeCall& c, uint8_t* scratch, uint32_t* status, cudaStream_t stream);
 
 }  // namespace smla

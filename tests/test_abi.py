@@ -36,7 +36,9 @@ def test_status_strings_and_version():
     assert L.smla_status_string(0) == b"SMLA_OK"
     assert L.smla_status_string(4) == b"SMLA_ERR_DEVICE_TIMEOUT"
     assert L.smla_status_string(99) == b"SMLA_UNKNOWN_STATUS"
-    assert L.smla_version() == 100
+    assert L.smla_version() == 101
+    assert L.smla_last_cuda_error() == 0
+    assert L.smla_last_cuda_error_string() == b"cudaSuccess"
 
 
 def test_workspace_bytes_arithmetic():

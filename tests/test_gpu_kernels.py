@@ -176,12 +176,13 @@ def test_softmax_scale_argument(smla):
     _check(w, softmax_scale=0.11)
 
 
-def test_bad_block_table_entry_is_skipped_and_flagged(smla, torch_cuda):
+@pytest.mark.parametrize("bad_entry", [10 ** 6, -5], ids=["past_cache", "negative"])
+def test_bad_block_table_entry_is_skipped_and_flagged(smla, torch_cuda, bad_entry):
     torch = torch_cuda
     w = W.Workload("badbt", batch=1, s_q=1, h_q=16, topk=64, seed=9, seqlens=(256,), index_mode="uniform")
     hi = PU.build_host_inputs(w)
     bt = hi.block_table.copy()
-    bt[0, 2] = 10 ** 6                                  # past the cache
+    bt[0, 2] = bad_entry                                # outside the cache
     d = PU.to_device(hi)
     d["block_table"] = torch.from_numpy(bt).cuda()
     import sparse_mla_decoding_b200 as m
@@ -249,3 +250,37 @@ def test_dequant_every_code_and_scale_range_is_exact(smla, torch_cuda):
     d["kvcache"] = torch.from_numpy(cache2).cuda()
     o2, _ = m.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"], sm, ns)
     assert np.isnan(o2[0, 0].float().cpu().numpy()).all()
+
+
+def test_flags_reach_callers_without_a_workspace(smla, torch_cuda):
+    """Calls that pass no workspace share one per device and stream; its status
+    word must report a skipped bad block-table entry, survive the buffer being
+    replaced by a larger one, and make check_device_status raise."""
+    torch = torch_cuda
+    import sparse_mla_decoding_b200 as m
+    w = W.Workload("badbt_cached", batch=1, s_q=1, h_q=16, topk=64, seed=19, seqlens=(256,), index_mode="uniform")
+    hi = PU.build_host_inputs(w)
+    d = PU.to_device(hi)
+    d["block_table"][0, 1] = -1
+    sm, ns = m.get_mla_metadata(d["cache_seqlens"], 64, 16, s_q=1)
+    m.reset_cached_workspace_status()
+    m.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"], sm, ns)
+    st, raw = m.cached_workspace_status()
+    assert st == 1 and raw & 2
+    # a larger call replaces the shared buffer; the flag is carried over
+    w2 = W.Workload("grow_cached", batch=8, s_q=1, h_q=128, topk=512, seed=20, seqlens=(1024,) * 8,
+                    index_mode="uniform")
+    hi2 = PU.build_host_inputs(w2)
+    d2 = PU.to_device(hi2)
+    sm2, ns2 = m.get_mla_metadata(d2["cache_seqlens"], 512, 128, s_q=1)
+    m.flash_mla_with_kvcache(d2["q"], d2["kvcache"], d2["block_table"], d2["cache_seqlens"], d2["indices"], sm2, ns2)
+    st, raw = m.cached_workspace_status()
+    assert st == 1 and raw & 2
+    with pytest.raises(m.SmlaError):
+        m.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"], sm, ns,
+                                 check_device_status=True)
+    m.reset_cached_workspace_status()
+    assert m.cached_workspace_status() == (0, 0)
+    d["block_table"][0, 1] = hi.block_table[0, 1]
+    m.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"], sm, ns,
+                             check_device_status=True)

@@ -5,8 +5,11 @@ runtimes, embedders that only hand over inputs and outputs, code where an
 allocation would synchronise or is not allowed): its split-KV scratch lives in
 a fixed 64 MiB array inside the library instead of a caller workspace.  Here it
 is called through the C ABI and its output is checked against the regular
-entry point's, under the parity tolerances, on two calls in a row (the array
-keeps the previous call's contents, which must not leak into the next).
+entry point's on two calls in a row (the array keeps the previous call's
+contents, which must not leak into the next): within the parity tolerances,
+and bit for bit, since the same kernels run with only the scratch pointer
+changed.  A flagged condition (a bad block-table entry) must reach the
+caller's status word through this entry point.
 This file is collected last on purpose.
 """
 import ctypes
@@ -75,7 +78,36 @@ def test_static_scratch_matches_regular_entry(w):
         assert rc == 0, f"call {call}: status {rc}"
         torch.cuda.synchronize()
         PU.compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref, f"{w.name} static-scratch call {call}")
+        assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref), f"call {call} differs from the regular entry"
     assert int(status.item()) == 0
+
+
+def test_static_scratch_reports_flags_to_the_caller():
+    """A valid index whose block-table entry lies outside the cache is skipped
+    and flagged; the flag must arrive in the caller's status word, and the
+    other rows must match the regular entry point bit for bit."""
+    import torch
+    import sparse_mla_decoding_b200 as smla
+    w = W.Workload("static_badbt", batch=2, s_q=1, h_q=64, topk=256, seed=43, seqlens=(512, 300),
+                   index_mode="uniform")
+    hi = PU.build_host_inputs(w)
+    d = PU.to_device(hi)
+    bt = d["block_table"].clone()
+    bt[0, 1] = -3
+    d["block_table"] = bt
+    sm, ns = smla.get_mla_metadata(d["cache_seqlens"], hi.indices.shape[2], w.h_q, s_q=w.s_q)
+    ws = smla.new_workspace(w.batch, w.s_q, w.h_q, hi.indices.shape[2], sm.shape[0])
+    o_ref, lse_ref = smla.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"],
+                                                 d["indices"], sm, ns, workspace=ws)
+    st, raw = smla.get_device_status(ws)
+    assert st == 1 and raw & 2
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o = torch.full_like(o_ref, float("nan"))
+    lse = torch.full_like(lse_ref, float("nan"))
+    assert _call_static(d, sm, ns, w, o, lse, status=status) == 0
+    torch.cuda.synchronize()
+    assert int(status.item()) & 2
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
 
 
 def test_static_scratch_rejects_oversized_calls():
