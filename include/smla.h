@@ -227,8 +227,13 @@ int smla_get_device_status(const void* workspace, int* status_out, uint32_t* raw
  *   Arguments as for smla_flash_mla_with_kvcache, without the workspace, plus
  *   status_out : device uint32 (may be NULL).  If given, the kernels OR their
  *                status flags (see smla_get_device_status) into it; the
- *                caller zeroes it.  If NULL, the flags go to the scratch
- *                header, which each call clears first and nothing reads back.
+ *                caller zeroes it and reads it after the call.  If NULL, the
+ *                flags go to the scratch header, which each call clears
+ *                first and which no API reads back: the caller then gives up
+ *                device-side error detection, and after such an error (a bad
+ *                block-table entry, inconsistent metadata, a wait that gave
+ *                up) o and lse may be built from incomplete or stale partials
+ *                while the call still returns SMLA_OK.
  * The scratch need is the same as smla_workspace_bytes(batch, s_q, h_q, topk,
  * num_sm_parts); a call that needs more returns SMLA_ERR_SCRATCH_LIMIT and
  * launches nothing.  Every call on a device shares the one array and it keeps
@@ -236,7 +241,9 @@ int smla_get_device_status(const void* workspace, int* status_out, uint32_t* raw
  * streams, other host threads) race on it and must be serialised by the
  * caller.  The first call on each device does a one-time set-up with that
  * device current (it looks up the array's device address and sets a kernel
- * attribute), so make that first call before any stream capture.
+ * attribute), repeated only if the device's CUDA context is re-created (for
+ * instance after cudaDeviceReset, which loads the module anew); make that
+ * first call before any stream capture.
  */
 int smla_flash_mla_with_kvcache_static_scratch(const void* q, const uint8_t* kvcache, int64_t num_blocks,
                                                const int32_t* block_table, int max_blocks,
