@@ -51,7 +51,23 @@ def parse():
     ap.add_argument("--copies", type=int, default=4, help="independent input copies rotated over the steps")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="skip the per-workload records of the other shapes and of the sparse-prefill entry")
     return ap.parse_args()
+
+
+def host_cpu():
+    """(logical cores, model name) of the host the CPU baseline runs on."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 0, model
 
 
 def valid_counts(idx: np.ndarray, seqlens: np.ndarray) -> np.ndarray:
@@ -224,7 +240,8 @@ def run_reference(args, w, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q, "topk": w.topk},
-        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": 1, "host_cores": host_cpu()[0],
+                         "cpu_model": host_cpu()[1], "kind": "oracle",
                          "sample": f"{tot_n} of {n_tok} query tokens per pass over {args.steps} steps "
                                    f"(single-threaded float64 C oracle)"},
         "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -236,8 +253,14 @@ def run_reference(args, w, rank, world):
 # our arm
 # ---------------------------------------------------------------------------
 
-def make_device_copy(w, device):
-    """Generator values -> device tensors; the cache rows are written by the library's own KV writer."""
+def make_device_copy(w, device, values="host"):
+    """Generator values -> device tensors; the cache rows are written by the library's own KV writer.
+
+    values="host" draws the cache values with the shared generator (the streams
+    the tests use); values="device" draws the same distributions (N(0,1), the
+    workload's outlier channels x8) with a seeded torch generator on the GPU,
+    which is much faster for the multi-GB caches.  Queries, lengths, block
+    tables and indices always come from the shared generator."""
     import torch
     import sparse_mla_decoding_b200 as smla
     from sparse_mla_decoding_b200 import workloads as W
@@ -245,11 +268,24 @@ def make_device_copy(w, device):
     rows = lay.num_blocks * W.BLOCK
     cache = torch.empty((lay.num_blocks, W.BLOCK, ROW), dtype=torch.uint8, device=device)
     flat = cache.view(rows, ROW)
-    for start, lat, rope in W.cache_values(w, rows, chunk_rows=W.GEN_CHUNK_ROWS * 4):
-        n = lat.shape[0]
-        dl = torch.from_numpy(lat.view(np.int16)).to(device).view(torch.bfloat16)
-        dr = torch.from_numpy(rope.view(np.int16)).to(device).view(torch.bfloat16)
-        smla.quantize_kv(dl, dr, flat[start:start + n])
+    if values == "host":
+        for start, lat, rope in W.cache_values(w, rows, chunk_rows=W.GEN_CHUNK_ROWS * 4):
+            n = lat.shape[0]
+            dl = torch.from_numpy(lat.view(np.int16)).to(device).view(torch.bfloat16)
+            dr = torch.from_numpy(rope.view(np.int16)).to(device).view(torch.bfloat16)
+            smla.quantize_kv(dl, dr, flat[start:start + n])
+    else:
+        gen = torch.Generator(device=device)
+        gen.manual_seed(int(w.seed) * 7919 + 11)
+        ch = torch.from_numpy(W.outlier_channels(w)).to(device)
+        step = 1 << 20
+        for start in range(0, rows, step):
+            n = min(step, rows - start)
+            lat = torch.randn((n, DV), generator=gen, device=device)
+            if ch.numel():
+                lat[:, ch] *= w.outlier_factor
+            rope = torch.randn((n, 64), generator=gen, device=device)
+            smla.quantize_kv(lat.to(torch.bfloat16), rope.to(torch.bfloat16), flat[start:start + n])
     unused = torch.from_numpy(W.unused_rows(lay)).to(device)
     flat[unused] = torch.from_numpy(W.POISON_ROW).to(device)
     idx = W.indices(w, lay.seqlens)
@@ -310,6 +346,186 @@ def reduce_over_ranks(times, work, device, world):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dist.all_reduce(s, op=dist.ReduceOp.SUM)
     return t.tolist(), s.tolist()
+
+
+def roofline(peaks, h_q, per_launch_flops, per_launch_bytes, launch_ms):
+    """Roofline of one launch: tensor-bound above the measured ridge, HBM-bound below it."""
+    intensity = (2.0 * h_q * (DQK + DV)) / ROW
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if intensity >= ridge:
+        achieved = per_launch_flops / (launch_ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"]}
+    achieved = per_launch_bytes / (launch_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"]}
+
+
+def timed(fn, n, stream, flush=None):
+    """Mean device time (ms) of fn() over n calls, with CUDA events on `stream`.
+
+    Without `flush` the calls run back to back between two events; with it,
+    every call is bracketed by its own events and flush() runs between calls,
+    outside the timed intervals."""
+    import torch
+    if flush is None:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for i in range(n):
+            fn(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    torch.cuda.synchronize()
+    for i in range(n):
+        flush()
+        evs[i][0].record(stream)
+        fn(i)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return float(np.mean([x.elapsed_time(y) for x, y in evs]))
+
+
+# How each extra record keeps a step's gathered rows from being served out of
+# L2 by an earlier timed step, and how its cache values are drawn.
+EXTRA_DECODE = (
+    ("tiny_h16_b2_topk64", 1, "host", "flush",
+     "one copy; L2 flushed (256 MB write) between individually timed calls"),
+    ("decode_h64_b128_sq2_topk2048", 1, "device", None,
+     "one copy: each step gathers 327 MB of rows from a 2.75 GB cache, both larger than the 126 MB L2"),
+    ("longctx_varlen_h128_b32_topk2048", 4, "device", None,
+     "inputs rotated over 4 independent copies (4 x 43 MB of rows per step, 4 x 1.5 GB caches) > 126 MB L2"),
+    ("prefill_shaped_h128_sq4096_topk2048", 1, "device", None,
+     "one copy: 604 MB of queries per step > 126 MB L2; the 43 MB cache itself is L2-resident by design "
+     "(each step reads it 128 times over), so its GB/s are L2 reads"),
+)
+
+
+def decode_record(w, n_copies, values, mode, l2_note, args, device, rank, world, peaks):
+    """The headline measurements (whole step, decode call, end to end) for one more workload."""
+    import torch
+    import sparse_mla_decoding_b200 as smla
+    stream = torch.cuda.current_stream(device)
+    copies = [make_device_copy(w.with_(seed=rank_seed(w, rank, c)), device, values) for c in range(n_copies)]
+    torch.cuda.synchronize()
+    flops = [step_flops(w.h_q, valid_counts(c["idx_host"], c["seqlens_host"])) for c in copies]
+    valid = [float(valid_counts(c["idx_host"], c["seqlens_host"]).sum()) for c in copies]
+    num_parts = smla.default_num_sm_parts(w.h_q, device)
+    ws = smla.new_workspace(w.batch, w.s_q, w.h_q, w.topk, num_parts, device)
+    outs = (torch.empty((w.batch, w.s_q, w.h_q, DV), dtype=torch.bfloat16, device=device),
+            torch.empty((w.batch, w.s_q, w.h_q), dtype=torch.float32, device=device))
+    metas = [smla.get_mla_metadata(c["cache_seqlens"], w.topk, w.h_q, num_parts, s_q=w.s_q) for c in copies]
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device) if mode == "flush" else None
+    flush = (lambda: flush_buf.fill_(1)) if flush_buf is not None else None
+
+    def step(i):
+        d = copies[i % n_copies]
+        sm, ns = smla.get_mla_metadata(d["cache_seqlens"], w.topk, w.h_q, num_parts, s_q=w.s_q)
+        smla.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"],
+                                    sm, ns, workspace=ws, out=outs)
+
+    def call(i):
+        d, (sm, ns) = copies[i % n_copies], metas[i % n_copies]
+        smla.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"],
+                                    sm, ns, workspace=ws, out=outs)
+
+    host = [dict(q=c["q"].cpu().pin_memory(), indices=c["indices"].cpu().pin_memory(),
+                 block_table=c["block_table"].cpu().pin_memory(), cache_seqlens=c["cache_seqlens"].cpu().pin_memory())
+            for c in copies]
+    dq, di = torch.empty_like(copies[0]["q"]), torch.empty_like(copies[0]["indices"])
+    dsl = torch.empty_like(copies[0]["cache_seqlens"])
+    dbt = [torch.empty_like(c["block_table"]) for c in copies]   # widths differ when lengths are drawn
+    ho = torch.empty(outs[0].shape, dtype=outs[0].dtype).pin_memory()
+    hl = torch.empty(outs[1].shape, dtype=outs[1].dtype).pin_memory()
+    h2d = int(np.mean([sum(h[k].numel() * h[k].element_size() for k in h) for h in host]))
+    d2h = ho.numel() * 2 + hl.numel() * 4
+
+    def e2e_step(i):
+        h, c = host[i % n_copies], copies[i % n_copies]
+        dq.copy_(h["q"], non_blocking=True)
+        di.copy_(h["indices"], non_blocking=True)
+        dbt[i % n_copies].copy_(h["block_table"], non_blocking=True)
+        dsl.copy_(h["cache_seqlens"], non_blocking=True)
+        sm, ns = smla.get_mla_metadata(dsl, w.topk, w.h_q, num_parts, s_q=w.s_q)
+        o, l = smla.flash_mla_with_kvcache(dq, c["kvcache"], dbt[i % n_copies], dsl, di, sm, ns, workspace=ws,
+                                           out=outs)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(l, non_blocking=True)
+
+    steps = max(args.steps // 2, 8)
+    for i in range(args.warmup):
+        step(i)
+        e2e_step(i)
+    step_ms = timed(step, steps, stream, flush)
+    call_ms = timed(call, steps, stream, flush)
+    e2e_ms = timed(e2e_step, steps, stream, flush)
+    status, raw = smla.get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status word set during the {w.name} record: {raw:#x}")
+    mean_f, mean_v = float(np.mean(flops)), float(np.mean(valid))
+    (step_ms, call_ms, e2e_ms), (f_all, v_all) = reduce_over_ranks([step_ms, call_ms, e2e_ms], [mean_f, mean_v],
+                                                                   device, world)
+    rec = {"value": f_all / (step_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": step_ms, "steps": steps,
+           "gathered_kv_gbs": v_all * ROW / (step_ms * 1e-3) / 1e9,
+           "roofline": dict(roofline(peaks, w.h_q, mean_f, mean_v * ROW, call_ms),
+                            kernel="splitkv_mla_kernel + combine_kernel (one decode call)", kernel_ms=call_ms,
+                            traffic=measured_traffic(w.name), peak_source=peaks["source"] + " (burst)"),
+           "e2e": {"value": f_all / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+                   "d2h_bytes_per_step": int(d2h)},
+           "config": {"workload": w.name, "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q, "topk": w.topk,
+                      "cache_values": "shared generator" if values == "host" else "seeded torch generator on the GPU",
+                      "l2": l2_note}}
+    del copies, host, ws, flush_buf
+    torch.cuda.empty_cache()
+    return rec
+
+
+def sparse_fwd_record(args, device, rank, world, peaks):
+    """flash_mla_sparse_fwd on the prefill-shaped workload: 4096 query tokens over one flat FP8 cache."""
+    import torch
+    import sparse_mla_decoding_b200 as smla
+    from sparse_mla_decoding_b200 import workloads as W
+    w = W.BY_NAME["prefill_shaped_h128_sq4096_topk2048"].with_(seed=rank_seed(W.PREFILL_SHAPED, rank, 0))
+    stream = torch.cuda.current_stream(device)
+    d = make_device_copy(w, device, "device")
+    s_kv = int(d["seqlens_host"][0])
+    # the flat cache holds logical token i at row i
+    pos = torch.arange(s_kv, device=device)
+    rows = d["block_table"][0].long()[pos // W.BLOCK] * W.BLOCK + pos % W.BLOCK
+    kv = d["kvcache"].view(-1, ROW).index_select(0, rows).contiguous()
+    q = d["q"].view(w.s_q, w.h_q, DQK)
+    idx = d["indices"].view(w.s_q, 1, w.topk)
+    f = step_flops(w.h_q, valid_counts(d["idx_host"], d["seqlens_host"]))
+    v = float(valid_counts(d["idx_host"], d["seqlens_host"]).sum())
+    parts = smla.default_num_sm_parts(w.h_q, device)
+    ws = smla.new_sparse_fwd_workspace(w.s_q, w.h_q, s_kv, w.topk, parts, device)
+    outs = (torch.empty((w.s_q, w.h_q, DV), dtype=torch.bfloat16, device=device),
+            torch.empty((w.s_q, w.h_q), dtype=torch.float32, device=device))
+
+    def call(i):
+        smla.flash_mla_sparse_fwd(q, kv, idx, num_sm_parts=parts, workspace=ws, out=outs)
+
+    for i in range(args.warmup):
+        call(i)
+    steps = max(args.steps // 5, 4)
+    ms = timed(call, steps, stream)
+    status, raw = smla.get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status word set during the sparse_fwd record: {raw:#x}")
+    (ms,), (f_all, v_all) = reduce_over_ranks([ms], [f, v], device, world)
+    rec = {"value": f_all / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "steps": steps,
+           "gathered_kv_gbs_l2": v_all * ROW / (ms * 1e-3) / 1e9,
+           "roofline": dict(roofline(peaks, w.h_q, f, v * ROW, ms),
+                            kernel="flash_mla_sparse_fwd (set-up + metadata + split kernel + combine)",
+                            peak_source=peaks["source"] + " (burst)"),
+           "config": {"api": "flash_mla_sparse_fwd", "s_q": w.s_q, "h_q": w.h_q, "s_kv": s_kv, "topk": w.topk,
+                      "indices": "causal, < 61440 + query position",
+                      "l2": "604 MB of queries per call > 126 MB L2; the 43 MB cache is L2-resident by design"}}
+    del d, kv, ws
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_ours(args, w, rank, world, local_rank):
@@ -428,25 +644,23 @@ def run_ours(args, w, rank, world, local_rank):
     # ---- reduce over ranks (max time, summed work) --------------------------
     (ms_total, e2e_ms, kern_ms), (tot_flops, tot_valid) = reduce_over_ranks(
         [ms_total, e2e_ms, kern_ms], [my_flops, my_valid], device, world)
+    peaks = load_peaks()
     if rank != 0:
+        # the other ranks take the same collective steps for the extra records
+        if not args.no_extra_workloads:
+            from sparse_mla_decoding_b200 import workloads as W
+            for name, n_copies, values, mode, note in EXTRA_DECODE:
+                if name != w.name:
+                    decode_record(W.BY_NAME[name], n_copies, values, mode, note, args, device, rank, world, peaks)
+            sparse_fwd_record(args, device, rank, world, peaks)
         return
 
-    peaks = load_peaks()
     tflops = tot_flops / (ms_total * 1e-3) / 1e12
     gbs = tot_valid * ROW / (ms_total * 1e-3) / 1e9
     # roofline of the decode call on this rank: per-launch algorithmic work / average launch duration
     per_launch_flops = float(np.mean(flops_per_copy))
     per_launch_bytes = float(np.mean(valid_per_copy)) * ROW
-    intensity = (2.0 * w.h_q * (DQK + DV)) / ROW
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if intensity >= ridge:
-        achieved = per_launch_flops / (kern_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"]}
-    else:
-        achieved = per_launch_bytes / (kern_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"]}
+    roof = roofline(peaks, w.h_q, per_launch_flops, per_launch_bytes, kern_ms)
     roof.update({"traffic": measured_traffic(w.name), "kernel": "splitkv_mla_kernel + combine_kernel (one decode call)",
                  "kernel_ms": kern_ms, "peak_source": peaks["source"] + " (burst)"})
 
@@ -470,9 +684,20 @@ def run_ours(args, w, rank, world, local_rank):
     if world == 1 and not args.no_cpu_baseline:
         hi = host_inputs(w.with_(seed=w.seed))
         f, t, n = cpu_oracle_sample(w, hi, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+        cores, model = host_cpu()
+        line["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": 1, "host_cores": cores,
+                                "cpu_model": model, "kind": "oracle",
                                 "sample": f"{n} of {w.batch * w.s_q} query tokens of the same workload, "
                                           f"{t:.1f} s single-threaded float64 C oracle"}
+    if not args.no_extra_workloads:
+        from sparse_mla_decoding_b200 import workloads as W
+        extra = {}
+        for name, n_copies, values, mode, note in EXTRA_DECODE:
+            if name == w.name:
+                continue
+            extra[name] = decode_record(W.BY_NAME[name], n_copies, values, mode, note, args, device, rank, world, peaks)
+        extra["sparse_fwd_prefill_shaped_h128_sq4096_topk2048"] = sparse_fwd_record(args, device, rank, world, peaks)
+        line["workloads"] = extra
     print(json.dumps(line), flush=True)
 
 
