@@ -83,6 +83,15 @@ def load(path: str) -> ctypes.CDLL:
     L.smo_combine.restype = None
     L.smo_sched_meta.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, c_i32p, c_i32p]
     L.smo_sched_meta.restype = ctypes.c_int
+    L.smo_sched_meta_varlen.argtypes = [ctypes.c_int, c_i32p, ctypes.c_int, c_i32p, c_i32p, c_i32p]
+    L.smo_sched_meta_varlen.restype = ctypes.c_int
+    L.smo_bf16_row.argtypes = [c_u8p, c_dp]
+    L.smo_bf16_row.restype = None
+    L.smo_dense_visible_len.argtypes = [ctypes.c_int32, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    L.smo_dense_visible_len.restype = ctypes.c_int32
+    L.smo_dense_decode_token.argtypes = [ctypes.c_int, c_u16p, c_u8p, ctypes.c_int, ctypes.c_int64, c_i32p,
+                                         ctypes.c_int, ctypes.c_int32, ctypes.c_double, c_dp, c_dp]
+    L.smo_dense_decode_token.restype = ctypes.c_int
     return L
 
 
@@ -286,6 +295,68 @@ def sparse_prefill(q_bits: np.ndarray, kv_rows: np.ndarray, indices: np.ndarray,
 
 
 # --------------------------------------------------------------------------
+# dense decode (every visible token; FP8 or BF16 cache rows)
+# --------------------------------------------------------------------------
+
+BF16_ROW_BYTES = 1152
+KV_FP8, KV_BF16 = 0, 1
+
+
+def bf16_row(row: np.ndarray) -> np.ndarray:
+    """A 1152-byte BF16 cache row -> the 576-wide key in float64."""
+    r = np.ascontiguousarray(row, dtype=np.uint8).reshape(-1)
+    assert r.size == BF16_ROW_BYTES
+    k = np.zeros(DQK, dtype=np.float64)
+    lib().smo_bf16_row(_ptr(r, ctypes.c_uint8), _ptr(k, ctypes.c_double))
+    return k
+
+
+def dense_visible_len(seqlen: int, s_q: int, t: int, causal: bool) -> int:
+    return int(lib().smo_dense_visible_len(int(seqlen), int(s_q), int(t), 1 if causal else 0))
+
+
+def dense_decode_token(q_bits: np.ndarray, kvcache: np.ndarray, kv_format: int, block_table_row: np.ndarray,
+                       length: int, softmax_scale: float = DEFAULT_SOFTMAX_SCALE):
+    """One query token over cache positions 0..length-1: kvcache [num_blocks,64,row] uint8 with
+    row = 656 (kv_format KV_FP8) or 1152 (KV_BF16) -> (o [h,512], lse [h])."""
+    qb = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    h = qb.shape[0]
+    row = BF16_ROW_BYTES if kv_format == KV_BF16 else ROW_BYTES
+    cache = kvcache if kvcache.flags["C_CONTIGUOUS"] else np.ascontiguousarray(kvcache)
+    num_blocks = cache.size // (BLOCK * row)
+    bt = np.ascontiguousarray(block_table_row, dtype=np.int32)
+    o = np.zeros((h, DV), dtype=np.float64)
+    lse = np.zeros(h, dtype=np.float64)
+    rc = lib().smo_dense_decode_token(h, _ptr(qb, ctypes.c_uint16), _ptr(cache.reshape(-1), ctypes.c_uint8),
+                                      int(kv_format), num_blocks, _ptr(bt, ctypes.c_int32), bt.shape[0], int(length),
+                                      float(softmax_scale), _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise ValueError("oracle: a position maps outside the block table or the cache")
+    return o, lse
+
+
+def dense_decode(q_bits: np.ndarray, kvcache: np.ndarray, kv_format: int, block_table: np.ndarray,
+                 cache_seqlens: np.ndarray, causal: bool, softmax_scale: float = DEFAULT_SOFTMAX_SCALE,
+                 tokens=None, threads: int = 1):
+    """Dense decode of a batch: q_bits [b,s_q,h,576] -> dict (b,t) -> (o, lse); each token single-threaded,
+    ``threads`` > 1 fans tokens out over host threads."""
+    b, s_q = q_bits.shape[0], q_bits.shape[1]
+    if tokens is None:
+        tokens = [(i, t) for i in range(b) for t in range(s_q)]
+    cache = np.ascontiguousarray(kvcache)
+
+    def one(bt_):
+        i, t = bt_
+        n = dense_visible_len(int(cache_seqlens[i]), s_q, t, causal)
+        return bt_, dense_decode_token(q_bits[i, t], cache, kv_format, block_table[i], n, softmax_scale)
+
+    if threads <= 1:
+        return dict(one(x) for x in tokens)
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        return dict(ex.map(one, tokens))
+
+
+# --------------------------------------------------------------------------
 # scheduler metadata
 # --------------------------------------------------------------------------
 
@@ -297,3 +368,27 @@ def sched_meta(R: int, n: int, P: int):
     if rc != 0:
         raise ValueError("oracle.sched_meta: invalid arguments")
     return sm, ns
+
+
+def sched_meta_varlen(n_tiles: np.ndarray, P: int):
+    """Scheduler metadata for per-request tile counts -> (sched_meta [P,8], num_splits [R+1], tile_prefix [R+1])."""
+    n = np.ascontiguousarray(n_tiles, dtype=np.int32)
+    R = n.shape[0]
+    sm = np.zeros((P, 8), dtype=np.int32)
+    ns = np.zeros(R + 1, dtype=np.int32)
+    tp = np.zeros(R + 1, dtype=np.int32)
+    rc = lib().smo_sched_meta_varlen(R, _ptr(n, ctypes.c_int32), P, _ptr(sm, ctypes.c_int32), _ptr(ns, ctypes.c_int32),
+                                     _ptr(tp, ctypes.c_int32))
+    if rc != 0:
+        raise ValueError("oracle.sched_meta_varlen: invalid arguments")
+    return sm, ns, tp
+
+
+def dense_tile_counts(cache_seqlens: np.ndarray, s_q: int, causal: bool) -> np.ndarray:
+    """Per request r = b * s_q + t of a dense decode: max(1, ceil(visible tokens / 64))."""
+    out = []
+    for sl in np.asarray(cache_seqlens):
+        for t in range(s_q):
+            n = dense_visible_len(int(sl), s_q, t, causal)
+            out.append(max(1, (n + BLOCK - 1) // BLOCK))
+    return np.asarray(out, dtype=np.int32)

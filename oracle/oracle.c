@@ -17,7 +17,8 @@
  *  [SRC-AL]    "deepseek-ai/FlashMLA" (agentlenshq project page), section
  *              技術的な詳細 (indices: -1 marks an entry the kernel ignores).
  *  [SRC-BLOG]  "FlashMLA：DeepSeek开源的高效MLA解码内核，专为NVIDIA Hopper GPU优化",
- *              section 主要功能特性 (paged KV cache with block size 64).
+ *              sections 主要功能特性 (paged KV cache with block size 64, BF16)
+ *              and 基础用法示例 (the dense decode call with causal=True).
  * The method as a whole: MQA with one KV head, d_qk = 576 (512 latent + 64
  * RoPE), d_v = 512 (the latent part), each query token attends to the top-k
  * cache rows its indices list; softmax_scale defaults to 1/sqrt(576); the
@@ -44,6 +45,7 @@
 #define SMO_BLOCK 64          /* paged-cache block size in tokens             */
 #define SMO_SCALE_OFF 512     /* byte offset of the 4 float32 scales          */
 #define SMO_ROPE_OFF 528      /* byte offset of the 64 bf16 RoPE values       */
+#define SMO_BF16_ROW_BYTES 1152  /* dense BF16 cache row: 576 bf16 values    */
 
 /* ------------------------------------------------------------------------ */
 /* Number formats                                                            */
@@ -306,6 +308,67 @@ int smo_sparse_decode_token(int h_q, const uint16_t* q_bf16, const uint8_t* kvca
 }
 
 /* ------------------------------------------------------------------------ */
+/* Dense decode: every visible cache token [SRC-BLOG 主要功能特性, 基础用法示例] */
+/* ------------------------------------------------------------------------ */
+
+/* A BF16 cache row holds the 576-wide key as 576 little-endian bf16 values
+ * (latent then RoPE); nothing is quantised. */
+void smo_bf16_row(const uint8_t* row, double* k)
+{
+    int i;
+    for (i = 0; i < SMO_DQK; ++i) k[i] = smo_bf16_to_double(smo_load_u16le(row + 2 * i));
+}
+
+/* Cache tokens visible to query token t of s_q new tokens of a request whose
+ * cache holds seqlen tokens.  The s_q tokens are the last s_q positions of the
+ * cache; with the causal mask token t sees positions 0 .. seqlen - s_q + t,
+ * without it every position.  Clamped to [0, seqlen]. */
+int32_t smo_dense_visible_len(int32_t seqlen, int s_q, int t, int causal)
+{
+    int64_t len = causal ? (int64_t)seqlen - (s_q - 1 - t) : (int64_t)seqlen;
+    if (len < 0) len = 0;
+    if (len > seqlen) len = seqlen;
+    return (int32_t)len;
+}
+
+/* One query token of dense decoding: attention over cache positions
+ * 0 .. len-1 of the request, row of position i = block_table_row[i/64] * 64 +
+ * i % 64.  kv_format 0: 656-byte FP8 rows (dequantised as for the sparse
+ * decode); 1: 1152-byte BF16 rows.  Returns 0, or -1 if a position maps
+ * outside the block table or the cache (its token is then left out). */
+int smo_dense_decode_token(int h_q, const uint16_t* q_bf16, const uint8_t* kvcache, int kv_format,
+                           int64_t num_blocks, const int32_t* block_table_row, int max_blocks, int32_t len,
+                           double softmax_scale, double* o, double* lse)
+{
+    int i, rc = 0;
+    const size_t row_bytes = kv_format ? SMO_BF16_ROW_BYTES : SMO_ROW_BYTES;
+    const int n = len > 0 ? len : 0;
+    double* q = (double*)malloc(sizeof(double) * (size_t)h_q * SMO_DQK);
+    double* K = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * SMO_DQK);
+    uint8_t* valid = (uint8_t*)malloc((size_t)(n > 0 ? n : 1));
+    for (i = 0; i < h_q * SMO_DQK; ++i) q[i] = smo_bf16_to_double(q_bf16[i]);
+    for (i = 0; i < n; ++i) {
+        int32_t blk = i / SMO_BLOCK;
+        int64_t phys;
+        valid[i] = 0;
+        if (blk >= max_blocks) { rc = -1; continue; }
+        phys = (int64_t)block_table_row[blk];
+        if (phys < 0 || phys >= num_blocks) { rc = -1; continue; }
+        {
+            const uint8_t* row = kvcache + (size_t)(phys * SMO_BLOCK + i % SMO_BLOCK) * row_bytes;
+            if (kv_format) smo_bf16_row(row, K + (size_t)i * SMO_DQK);
+            else smo_dequantize_row(row, K + (size_t)i * SMO_DQK);
+        }
+        valid[i] = 1;
+    }
+    smo_attend(h_q, q, n, K, valid, softmax_scale, o, lse, NULL);
+    free(q);
+    free(K);
+    free(valid);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
 /* LSE-weighted combine of split partials [SRC-WALK 合并与性能账本]          */
 /* ------------------------------------------------------------------------ */
 
@@ -382,6 +445,62 @@ int smo_sched_meta(int R, int n, int P, int32_t* sched_meta, int32_t* num_splits
         m[2] = (int32_t)(g1 / n);
         m[3] = (int32_t)(g1 % n);
         m[4] = num_splits[m[0]] + p - (int32_t)((((int64_t)m[0]) * n) / L);
+        m[5] = 0;
+    }
+    return 0;
+}
+
+/* The same division of work when requests have different numbers of tiles
+ * (dense decode: n[r] = ceil(visible tokens / 64), at least 1, so every
+ * request has a tile and gets its (o, lse) written).  tile_prefix[r] is the
+ * number of tiles before request r (length R + 1); the G = tile_prefix[R]
+ * tiles in (request, tile) order are cut into P ranges of L = ceil(G / P);
+ * part p covers global tiles [p L, min((p+1) L, G)).  A request's parts are
+ * first(r) = tile_prefix[r] / L .. last(r) = (tile_prefix[r+1] - 1) / L, and
+ * sched_meta / num_splits have the meaning of smo_sched_meta with tile
+ * positions counted within each request.  Returns -1 for a tile count < 1. */
+int smo_sched_meta_varlen(int R, const int32_t* n, int P, int32_t* sched_meta, int32_t* num_splits,
+                          int32_t* tile_prefix)
+{
+    int64_t total, L;
+    int r, p;
+    if (R < 0 || P < 1) return -1;
+    tile_prefix[0] = 0;
+    for (r = 0; r < R; ++r) {
+        if (n[r] < 1) return -1;
+        tile_prefix[r + 1] = tile_prefix[r] + n[r];
+    }
+    total = tile_prefix[R];
+    L = total > 0 ? (total + P - 1) / P : 1;
+    num_splits[0] = 0;
+    for (r = 0; r < R; ++r) {
+        int64_t first = (int64_t)tile_prefix[r] / L;
+        int64_t last = ((int64_t)tile_prefix[r + 1] - 1) / L;
+        num_splits[r + 1] = num_splits[r] + (int32_t)(last - first + 1);
+    }
+    for (p = 0; p < P; ++p) {
+        int32_t* m = sched_meta + (size_t)p * 8;
+        int64_t g0 = (int64_t)p * L;
+        int64_t g1 = (int64_t)(p + 1) * L;
+        int i, rb, re;
+        for (i = 0; i < 8; ++i) m[i] = 0;
+        if (g0 >= total) { m[5] = 1; continue; }
+        if (g1 > total) g1 = total;
+        /* the request holding global tile g0: the last r with tile_prefix[r] <= g0 */
+        rb = 0;
+        while (rb + 1 < R && tile_prefix[rb + 1] <= g0) ++rb;
+        /* the exclusive end: request R with tile 0 when g1 reaches the total */
+        if (g1 == total) {
+            re = R;
+        } else {
+            re = rb;
+            while (re + 1 < R && tile_prefix[re + 1] <= g1) ++re;
+        }
+        m[0] = rb;
+        m[1] = (int32_t)(g0 - tile_prefix[rb]);
+        m[2] = re;
+        m[3] = (re == R) ? 0 : (int32_t)(g1 - tile_prefix[re]);
+        m[4] = num_splits[rb] + p - (int32_t)((int64_t)tile_prefix[rb] / L);
         m[5] = 0;
     }
     return 0;

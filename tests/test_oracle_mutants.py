@@ -45,7 +45,21 @@ MUTANTS = [
      "int64_t last = ((int64_t)(r + 1) * n) / L;"),
     ("sched first slot offset dropped",
      "m[4] = num_splits[m[0]] + p - (int32_t)((((int64_t)m[0]) * n) / L);", "m[4] = num_splits[m[0]];"),
-    ("sched tiles per part floor", "L = total > 0 ? (total + P - 1) / P : 1;", "L = total > 0 ? total / P + (total < P) : 1;"),
+    ("sched tiles per part floor", "L = total > 0 ? (total + P - 1) / P : 1;\n    num_splits[0] = 0;\n    for (r = 0; r < R; ++r) {\n        int64_t first = ((int64_t)r * n) / L;",
+     "L = total > 0 ? total / P + (total < P) : 1;\n    num_splits[0] = 0;\n    for (r = 0; r < R; ++r) {\n        int64_t first = ((int64_t)r * n) / L;"),
+    ("causal visible length off by one", "int64_t len = causal ? (int64_t)seqlen - (s_q - 1 - t) : (int64_t)seqlen;",
+     "int64_t len = causal ? (int64_t)seqlen - (s_q - t) : (int64_t)seqlen;"),
+    ("bf16 row read shifted", "k[i] = smo_bf16_to_double(smo_load_u16le(row + 2 * i));",
+     "k[i] = smo_bf16_to_double(smo_load_u16le(row + 2 * i + 2));"),
+    ("dense bf16 row stride of the latent only", "const size_t row_bytes = kv_format ? SMO_BF16_ROW_BYTES : SMO_ROW_BYTES;",
+     "const size_t row_bytes = kv_format ? 1024 : SMO_ROW_BYTES;"),
+    ("dense row within block", "(size_t)(phys * SMO_BLOCK + i % SMO_BLOCK) * row_bytes",
+     "(size_t)(phys * SMO_BLOCK + i % 32) * row_bytes"),
+    ("varlen last part off by one", "int64_t last = ((int64_t)tile_prefix[r + 1] - 1) / L;",
+     "int64_t last = ((int64_t)tile_prefix[r + 1]) / L;"),
+    ("varlen first tile not relative to its request", "m[1] = (int32_t)(g0 - tile_prefix[rb]);", "m[1] = (int32_t)g0;"),
+    ("varlen end request search stops early", "while (re + 1 < R && tile_prefix[re + 1] <= g1) ++re;",
+     "while (re + 1 < R && tile_prefix[re + 1] < g1) ++re;"),
 ]
 
 
@@ -56,6 +70,9 @@ def _pin_functions():
             continue
         if name == "test_sched_meta_brute_force":
             for args in [(64, 32, 148), (7, 3, 5), (5, 7, 35), (13, 2, 3), (3, 100, 7)]:
+                out.append((f"{name}{args}", lambda fn=fn, args=args: fn(*args)))
+        elif name == "test_sched_meta_varlen_brute_force":
+            for args in [([3, 1, 5, 2], 4), ([7, 1, 1, 1, 30, 2], 5), ([9, 9], 7), ([128] * 64, 148)]:
                 out.append((f"{name}{args}", lambda fn=fn, args=args: fn(*args)))
         else:
             out.append((name, fn))

@@ -451,3 +451,150 @@ def test_sched_meta_rejects_bad_arguments():
         oracle.sched_meta(4, 0, 8)
     with pytest.raises(ValueError):
         oracle.sched_meta(4, 2, 0)
+
+
+# --------------------------------------------------------------------------
+# dense decode: every visible token, FP8 or BF16 cache rows
+# --------------------------------------------------------------------------
+
+def test_bf16_row_matches_torch_cast():
+    import torch
+    rng = np.random.default_rng(51)
+    vals = np.concatenate([rng.standard_normal(500) * 10.0 ** rng.integers(-30, 30, 500), [0.0, -0.0, 1e38, -3e-39],
+                           rng.standard_normal(72)])[:576]
+    bits = _bits(vals)
+    row = bits.astype("<u2").tobytes()
+    k = oracle.bf16_row(np.frombuffer(row, np.uint8))
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).double().numpy()
+    assert np.array_equal(k, ref)
+
+
+def test_dense_visible_len_closed_forms():
+    for sl, s_q in [(100, 1), (100, 4), (3, 4), (0, 2), (64, 64)]:
+        for t in range(s_q):
+            assert oracle.dense_visible_len(sl, s_q, t, False) == sl
+            assert oracle.dense_visible_len(sl, s_q, t, True) == max(0, min(sl, sl - s_q + 1 + t))
+        # the last new token sees the whole cache; token t sees one more position than token t-1
+        if sl >= s_q:
+            assert oracle.dense_visible_len(sl, s_q, s_q - 1, True) == sl
+            assert [oracle.dense_visible_len(sl, s_q, t, True) for t in range(s_q)] == list(range(sl - s_q + 1, sl + 1))
+
+
+def test_dense_fp8_equals_sparse_decode_over_every_position():
+    """Dense decode is the sparse decode whose index list is every visible position."""
+    rng = np.random.default_rng(52)
+    nb, seqlen = 5, 300
+    lat = _bits(rng.standard_normal((nb * 64, DV)) * 3)
+    rope = _bits(rng.standard_normal((nb * 64, 64)))
+    cache = oracle.quantize_tokens(lat, rope).reshape(nb, 64, 656)
+    bt = rng.permutation(nb).astype(np.int32)
+    q_bits = _bits(rng.standard_normal((32, DQK)))
+    for n in (1, 63, 64, 65, 300):
+        o, lse = oracle.dense_decode_token(q_bits, cache, oracle.KV_FP8, bt, n)
+        o2, lse2 = oracle.sparse_decode_token(q_bits, cache, bt, seqlen, np.arange(n, dtype=np.int32))
+        assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+
+
+def _bf16_cache(rng, nb, perm):
+    """A paged BF16 cache (rows of 576 bf16 values) and its logical key matrix."""
+    logical = _bits(rng.standard_normal((nb * 64, DQK)))
+    Kl = oracle.bf16_bits_to_f64(logical)
+    phys = np.zeros_like(logical)
+    for lb in range(nb):
+        phys[perm[lb] * 64:(perm[lb] + 1) * 64] = logical[lb * 64:(lb + 1) * 64]
+    return np.frombuffer(phys.astype("<u2").tobytes(), np.uint8).reshape(nb, 64, 1152), Kl
+
+
+def test_dense_bf16_equals_textbook_over_visible_tokens():
+    rng = np.random.default_rng(53)
+    nb = 4
+    perm = rng.permutation(nb)
+    cache, Kl = _bf16_cache(rng, nb, perm)
+    q_bits = _bits(rng.standard_normal((16, DQK)))
+    q = oracle.bf16_bits_to_f64(q_bits)
+    for n in (1, 64, 130, 256):
+        o, lse = oracle.dense_decode_token(q_bits, cache, oracle.KV_BF16, perm.astype(np.int32), n)
+        o_ref, lse_ref = _textbook(q, Kl[:n], 1.0 / 24.0)
+        assert _close(o, o_ref) and _close(lse, lse_ref)
+
+
+def test_dense_batch_driver_applies_the_causal_mask():
+    rng = np.random.default_rng(54)
+    nb = 3
+    perm = rng.permutation(nb)
+    cache, Kl = _bf16_cache(rng, nb, perm)
+    s_q, seqlen = 3, 150
+    q_bits = _bits(rng.standard_normal((1, s_q, 8, DQK)))
+    bt = perm.astype(np.int32).reshape(1, -1)
+    for causal in (False, True):
+        out = oracle.dense_decode(q_bits, cache, oracle.KV_BF16, bt, np.array([seqlen]), causal)
+        for t in range(s_q):
+            n = seqlen - (s_q - 1 - t) if causal else seqlen
+            o_ref, lse_ref = _textbook(oracle.bf16_bits_to_f64(q_bits[0, t]), Kl[:n], 1.0 / 24.0)
+            assert _close(out[(0, t)][0], o_ref) and _close(out[(0, t)][1], lse_ref)
+
+
+def test_dense_zero_visible_tokens_gives_zero_and_minus_inf():
+    rng = np.random.default_rng(55)
+    cache, _ = _bf16_cache(rng, 1, np.array([0]))
+    o, lse = oracle.dense_decode_token(_bits(rng.standard_normal((4, DQK))), cache, oracle.KV_BF16,
+                                       np.array([0], np.int32), 0)
+    assert (o == 0).all() and np.isneginf(lse).all()
+
+
+def _brute_sched_varlen(n, P):
+    """Enumerate tiles one by one, filling parts of L tiles in (request, tile) order."""
+    total = int(np.sum(n))
+    L = -(-total // P) if total else 1
+    owner, g = {}, 0
+    for r, nr in enumerate(n):
+        for t in range(nr):
+            owner[(r, t)] = g // L
+            g += 1
+    parts = {p: sorted(k for k, v in owner.items() if v == p) for p in range(P)}
+    return L, owner, parts
+
+
+@pytest.mark.parametrize("n,P", [([3, 1, 5, 2], 4), ([1], 148), ([128] * 64, 148), ([7, 1, 1, 1, 30, 2], 5),
+                                 ([2048] * 2 + [64] * 30, 74), ([1] * 300, 148), ([4, 4, 4], 3), ([9, 9], 7)])
+def test_sched_meta_varlen_brute_force(n, P):
+    sm, ns, tp = oracle.sched_meta_varlen(np.array(n), P)
+    assert list(tp) == [0] + list(np.cumsum(n))
+    L, owner, parts = _brute_sched_varlen(n, P)
+    S = [len({owner[(r, t)] for t in range(nr)}) for r, nr in enumerate(n)]
+    assert ns[0] == 0 and list(np.diff(ns)) == S
+    covered = set()
+    for p in range(P):
+        tiles = parts[p]
+        if not tiles:
+            assert sm[p, 5] == 1 and (sm[p, :5] == 0).all()
+            continue
+        assert sm[p, 5] == 0 and (sm[p, 0], sm[p, 1]) == tiles[0]
+        last = tiles[-1]
+        end = (last[0], last[1] + 1) if last[1] + 1 < n[last[0]] else (last[0] + 1, 0)
+        assert (sm[p, 2], sm[p, 3]) == end
+        r0 = tiles[0][0]
+        parts_of_r0 = sorted({owner[(r0, t)] for t in range(n[r0])})
+        assert sm[p, 4] == ns[r0] + parts_of_r0.index(p)
+        covered.update(tiles)
+        assert len(tiles) <= L
+    assert covered == set(owner)
+
+
+def test_sched_meta_varlen_equals_uniform_for_equal_counts():
+    for R, k, P in [(64, 32, 148), (7, 3, 5), (256, 32, 148), (5, 7, 36)]:
+        sm, ns, _ = oracle.sched_meta_varlen(np.full(R, k), P)
+        sm_u, ns_u = oracle.sched_meta(R, k, P)
+        assert np.array_equal(sm, sm_u) and np.array_equal(ns, ns_u)
+
+
+def test_sched_meta_varlen_rejects_empty_requests():
+    with pytest.raises(ValueError):
+        oracle.sched_meta_varlen(np.array([2, 0, 1]), 4)
+
+
+def test_dense_tile_counts():
+    assert list(oracle.dense_tile_counts(np.array([1, 64, 65, 0]), 1, False)) == [1, 1, 2, 1]
+    # causal: token t of 3 sees seqlen - 2 + t positions: 126..128 -> 2, 2, 2 tiles; 128..130 -> 2, 3, 3
+    assert list(oracle.dense_tile_counts(np.array([128]), 3, True)) == [2, 2, 2]
+    assert list(oracle.dense_tile_counts(np.array([130]), 3, True)) == [2, 3, 3]
