@@ -152,6 +152,64 @@ int smla_flash_mla_with_kvcache(const void* q, const uint8_t* kvcache, int64_t n
                                 int num_sm_parts, float softmax_scale, int batch, int s_q, int h_q, int topk,
                                 void* o, float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Row formats of a dense-decode cache. */
+#define SMLA_KV_FP8 0           /* 656-byte rows as for the sparse decode                       */
+#define SMLA_KV_BF16 1          /* 1152-byte rows: the 576-wide key as bf16 (latent, then RoPE) */
+
+/*
+ * Scheduler metadata of a dense decode ("FlashMLA：DeepSeek开源的高效MLA解码内核…",
+ * sections 主要功能特性 and 基础用法示例: get_mla_metadata from the cache lengths,
+ * then flash_mla_with_kvcache with causal=True; "FlashMLA 注意力内核源码走读…",
+ * section 调度: the work is spread evenly over the SMs before the main kernel).
+ * Request r = b * s_q + t attends to the len_r visible tokens of batch entry
+ * b: len_r = cache_seqlens[b], or with the causal mask cache_seqlens[b] -
+ * (s_q - 1 - t) (the s_q new tokens are the last s_q positions of the cache),
+ * at least 0.  Its work is n_r = max(1, ceil(len_r / 64)) tiles, so the split
+ * follows the lengths: tile_prefix[r] = tiles before request r (tile_prefix[R]
+ * = the total, which must stay below 2^31), then the tiles in (request, tile)
+ * order are cut into num_sm_parts ranges of L = ceil(total / P) as for
+ * smla_get_mla_metadata, with tile positions counted within each request.
+ *   cache_seqlens : device int32 [batch]
+ *   sched_meta    : device int32 [num_sm_parts][8], written (16-byte aligned)
+ *   num_splits    : device int32 [batch*s_q + 1], written
+ *   tile_prefix   : device int32 [batch*s_q + 1], written
+ * Launches one CTA on `stream`; reusable while cache_seqlens, s_q, causal and
+ * num_sm_parts stay the same.
+ */
+int smla_get_mla_metadata_dense(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int causal,
+                                int num_sm_parts, int32_t* sched_meta, int32_t* num_splits, int32_t* tile_prefix,
+                                void* stream);
+
+/*
+ * Dense MLA decode: every query token attends to all its visible cache tokens
+ * ("FlashMLA：DeepSeek开源的高效MLA解码内核…", sections 主要功能特性 (paged cache
+ * with 64-token blocks, BF16) and 基础用法示例 (flash_mla_with_kvcache with
+ * causal=True)).  The same split kernel and combine as the sparse decode run
+ * with the index list of request r taken to be 0 .. len_r - 1 (len_r as in
+ * smla_get_mla_metadata_dense), made in the kernel instead of read from
+ * memory.  With kv_format SMLA_KV_FP8 the rows are the 656-byte FP8 rows of
+ * the sparse decode; with SMLA_KV_BF16 they are 1152-byte rows of 576 bf16
+ * values, used as they are.
+ *   q             : device bf16 [batch][s_q][h_q][576]
+ *   kvcache       : device uint8 [num_blocks][64][656 or 1152] (16-byte aligned)
+ *   block_table   : device int32 [batch][max_blocks]
+ *   cache_seqlens : device int32 [batch]
+ *   sched_meta, num_splits, tile_prefix : from smla_get_mla_metadata_dense
+ *                   with the same batch, s_q, causal and num_sm_parts
+ *   causal        : 0 or 1, as for the metadata
+ *   o, lse, workspace : as for smla_flash_mla_with_kvcache (the workspace
+ *                   size is smla_workspace_bytes(batch, s_q, h_q, 1,
+ *                   num_sm_parts))
+ * A visible position whose block lies outside block_table or the cache is
+ * skipped and flags the workspace status word, as in the sparse decode.
+ */
+int smla_flash_mla_dense_with_kvcache(const void* q, const uint8_t* kvcache, int kv_format, int64_t num_blocks,
+                                      const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                                      const int32_t* sched_meta, const int32_t* num_splits,
+                                      const int32_t* tile_prefix, int num_sm_parts, float softmax_scale, int causal,
+                                      int batch, int s_q, int h_q, void* o, float* lse, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
 /*
  * Sparse attention of many query tokens over one flat (unpaged) FP8 cache
  * ("deepseek-ai/FlashMLA" (agentlenshq), section 使用方法 item 2:

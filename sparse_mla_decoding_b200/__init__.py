@@ -65,6 +65,11 @@ def lib() -> ctypes.CDLL:
             L.smla_flash_mla_with_kvcache.argtypes = [vp, vp, i64, vp, i32, vp, vp, vp, vp, i32, f32, i32, i32, i32,
                                                       i32, vp, vp, vp, sz, vp]
             L.smla_flash_mla_with_kvcache.restype = i32
+            L.smla_get_mla_metadata_dense.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+            L.smla_get_mla_metadata_dense.restype = i32
+            L.smla_flash_mla_dense_with_kvcache.argtypes = [vp, vp, i32, i64, vp, i32, vp, vp, vp, vp, i32, f32, i32,
+                                                            i32, i32, i32, vp, vp, vp, sz, vp]
+            L.smla_flash_mla_dense_with_kvcache.restype = i32
             L.smla_flash_mla_sparse_fwd.argtypes = [vp, vp, i64, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
             L.smla_flash_mla_sparse_fwd.restype = i32
             L.smla_sparse_fwd_workspace_bytes.argtypes = [i32, i32, i64, i32, i32]
@@ -264,6 +269,100 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
     _check(rc, "smla_flash_mla_with_kvcache")
     if check_device_status:
         _raise_on_flags(workspace, "smla_flash_mla_with_kvcache")
+    return o, lse
+
+
+KV_FP8, KV_BF16 = 0, 1
+BF16_ROW_BYTES = 1152
+
+
+def get_mla_metadata_dense(cache_seqlens: torch.Tensor, h_q: int, s_q: int = 1, causal: bool = True,
+                           num_sm_parts: Optional[int] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Scheduler metadata of a dense decode, split by the requests' visible lengths.
+
+    Returns (sched_meta int32 [num_sm_parts, 8], num_splits int32 [b*s_q + 1],
+    tile_prefix int32 [b*s_q + 1]); reusable across layers while the lengths stay.
+    """
+    _require(cache_seqlens.is_cuda and cache_seqlens.dtype == torch.int32 and cache_seqlens.dim() == 1,
+             "cache_seqlens must be a 1-D int32 CUDA tensor")
+    dev = cache_seqlens.device
+    if num_sm_parts is None:
+        num_sm_parts = default_num_sm_parts(h_q, dev)
+    R = cache_seqlens.shape[0] * s_q
+    sched_meta = torch.empty((num_sm_parts, 8), dtype=torch.int32, device=dev)
+    num_splits = torch.empty((R + 1,), dtype=torch.int32, device=dev)
+    tile_prefix = torch.empty((R + 1,), dtype=torch.int32, device=dev)
+    rc = lib().smla_get_mla_metadata_dense(_ptr(cache_seqlens.contiguous()), cache_seqlens.shape[0], int(s_q), int(h_q),
+                                           1 if causal else 0, int(num_sm_parts), _ptr(sched_meta), _ptr(num_splits),
+                                           _ptr(tile_prefix), _stream(dev))
+    _check(rc, "smla_get_mla_metadata_dense")
+    return sched_meta, num_splits, tile_prefix
+
+
+def _kv_format(kvcache: torch.Tensor) -> int:
+    if kvcache.dtype == torch.uint8 and kvcache.shape[-1] == KV_ROW_BYTES:
+        return KV_FP8
+    if kvcache.dtype == torch.uint8 and kvcache.shape[-1] == BF16_ROW_BYTES:
+        return KV_BF16
+    if kvcache.dtype == torch.bfloat16 and kvcache.shape[-1] == D_QK:
+        return KV_BF16
+    raise ValueError("kvcache must be uint8 [..., 656] (FP8 rows), or bf16 [..., 576] / uint8 [..., 1152] (BF16 rows)")
+
+
+def flash_mla_dense_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: torch.Tensor,
+                                 cache_seqlens: torch.Tensor, sched_meta: torch.Tensor, num_splits: torch.Tensor,
+                                 tile_prefix: torch.Tensor, causal: bool = True,
+                                 softmax_scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
+                                 out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                                 check_device_status: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Dense MLA decode: every query token attends to all its visible cache tokens.
+
+    q: bf16 [b, s_q, h_q, 576]; kvcache: paged [num_blocks, 64, (1,) row] with FP8
+    rows (uint8, 656 bytes) or BF16 rows (bf16 576 values, or uint8 1152 bytes);
+    block_table: int32 [b, max_blocks]; cache_seqlens: int32 [b]; sched_meta /
+    num_splits / tile_prefix from get_mla_metadata_dense with the same lengths,
+    s_q and causal.  With causal=True token t of s_q sees the first
+    seqlen - (s_q - 1 - t) cache positions.  Returns (o bf16 [b, s_q, h_q, 512],
+    lse float32 [b, s_q, h_q]).
+    """
+    _require(q.is_cuda and q.dtype == torch.bfloat16 and q.dim() == 4 and q.shape[-1] == D_QK,
+             "q must be a bf16 CUDA tensor [b, s_q, h_q, 576]")
+    b, s_q, h_q, _ = q.shape
+    fmt = _kv_format(kvcache)
+    _require(kvcache.shape[1] == BLOCK_SIZE and kvcache.is_contiguous(), "kvcache must be contiguous [num_blocks, 64, ...]")
+    _require(block_table.dtype == torch.int32 and block_table.dim() == 2 and block_table.shape[0] == b,
+             "block_table must be int32 [b, max_blocks]")
+    _require(cache_seqlens.dtype == torch.int32 and tuple(cache_seqlens.shape) == (b,),
+             "cache_seqlens must be int32 [b]")
+    _require(sched_meta.dtype == torch.int32 and sched_meta.dim() == 2 and sched_meta.shape[1] == 8,
+             "sched_meta must be int32 [num_sm_parts, 8]")
+    for name, t in (("num_splits", num_splits), ("tile_prefix", tile_prefix)):
+        _require(t.dtype == torch.int32 and tuple(t.shape) == (b * s_q + 1,), f"{name} must be int32 [b*s_q + 1]")
+    for name, t in (("kvcache", kvcache), ("block_table", block_table), ("cache_seqlens", cache_seqlens),
+                    ("sched_meta", sched_meta), ("num_splits", num_splits), ("tile_prefix", tile_prefix)):
+        _require(t.is_cuda and t.device == q.device, f"{name} must be on {q.device}")
+        _require(t.is_contiguous(), f"{name} must be contiguous")
+    q = q.contiguous()
+    num_sm_parts = sched_meta.shape[0]
+    dev = q.device
+    nbytes = workspace_bytes(b, s_q, h_q, 1, num_sm_parts)
+    if workspace is None:
+        workspace = _cached_workspace(dev, nbytes)
+    _require(workspace.is_cuda and workspace.numel() * workspace.element_size() >= nbytes,
+             f"workspace needs {nbytes} bytes")
+    if out is None:
+        o = torch.empty((b, s_q, h_q, D_V), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((b, s_q, h_q), dtype=torch.float32, device=dev)
+    else:
+        o, lse = out
+    scale = -1.0 if softmax_scale is None else float(softmax_scale)
+    rc = lib().smla_flash_mla_dense_with_kvcache(
+        _ptr(q), _ptr(kvcache), fmt, kvcache.shape[0], _ptr(block_table), block_table.shape[1], _ptr(cache_seqlens),
+        _ptr(sched_meta), _ptr(num_splits), _ptr(tile_prefix), num_sm_parts, scale, 1 if causal else 0, b, s_q, h_q,
+        _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
+    _check(rc, "smla_flash_mla_dense_with_kvcache")
+    if check_device_status:
+        _raise_on_flags(workspace, "smla_flash_mla_dense_with_kvcache")
     return o, lse
 
 

@@ -195,6 +195,15 @@ __device__ __forceinline__ void tmem_ld16x2_32(uint32_t taddr, uint32_t (&r)[32]
 
 // Store counterparts of the 16x32bx2 shape: thread i writes lane
 // (base + i % 16), columns [col + N (i / 16), col + N (i / 16) + N) for .xN.
+// The .x8 form takes the offset of the second half as `half_off` columns:
+// thread i writes [col + half_off (i / 16), + 8).
+template <int kHalfOff>
+__device__ __forceinline__ void tmem_st16x2_8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.16x32bx2.x8.b32 [%0], %9, {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "n"(kHalfOff)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16x2_16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 16, "

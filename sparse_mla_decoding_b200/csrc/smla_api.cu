@@ -16,6 +16,8 @@
 
 namespace smla {
 __global__ void sched_meta_kernel(int R, int n, int P, int32_t* sched_meta, int32_t* num_splits);
+__global__ void sched_meta_dense_kernel(const int32_t* seqlens, int batch, int s_q, int causal, int P,
+                                        int32_t* sched_meta, int32_t* num_splits, int32_t* tile_prefix);
 __global__ void combine_kernel(const int32_t* num_splits, const float* o_accum, const float* lse_accum, int h_q,
                                int max_splits, __nv_bfloat16* o, float* lse);
 __global__ void quantize_kv_kernel(const __nv_bfloat16* latent, const __nv_bfloat16* rope, int64_t n_tokens,
@@ -98,8 +100,11 @@ int check_decode_call(const DecodeCall& c) {
       c.num_blocks > (int64_t)(0x7FFFFFFF / SMLA_BLOCK_SIZE))
     return SMLA_ERR_INVALID_ARGUMENT;
   if (c.batch == 0) return SMLA_OK;
-  if (!c.q || !c.kvcache || !c.block_table || !c.cache_seqlens || !c.indices || !c.sched_meta || !c.num_splits ||
-      !c.o || !c.lse)
+  const bool dense = c.kv_mode != kSparseFp8;
+  if (!c.q || !c.kvcache || !c.block_table || !c.cache_seqlens || (!dense && !c.indices) || !c.sched_meta ||
+      !c.num_splits || (dense && !c.tile_prefix) || !c.o || !c.lse)
+    return SMLA_ERR_INVALID_ARGUMENT;
+  if (c.kv_mode < kSparseFp8 || c.kv_mode > kDenseBf16 || (dense && c.causal != 0 && c.causal != 1))
     return SMLA_ERR_INVALID_ARGUMENT;
   if (!aligned(c.q, 16) || !aligned(c.kvcache, 16) || !aligned(c.o, 16) || !aligned(c.sched_meta, 16))
     return SMLA_ERR_INVALID_ARGUMENT;
@@ -140,12 +145,15 @@ int launch_decode(const DecodeCall& c, uint8_t* scratch, uint32_t* status, cudaS
   p.max_blocks = c.max_blocks;
   p.seqlens = c.cache_seqlens;
   p.indices = c.indices;
+  p.tile_prefix = c.tile_prefix;
+  p.kv_mode = c.kv_mode;
+  p.causal = c.causal;
   p.sched_meta = c.sched_meta;
   p.num_splits = c.num_splits;
   p.s_q = c.s_q;
   p.h_q = c.h_q;
   p.topk = c.topk;
-  p.n_tiles = (int)n_tiles_of(c.topk);
+  p.n_tiles = c.tile_prefix ? 0 : (int)n_tiles_of(c.topk);
   p.num_parts = c.num_sm_parts;
   p.num_requests = (int)R;
   p.max_splits = (int)(R + c.num_sm_parts);
@@ -239,6 +247,49 @@ int smla_flash_mla_with_kvcache(const void* q, const uint8_t* kvcache, int64_t n
   const smla::DecodeCall c{q,          kvcache, num_blocks, block_table, max_blocks, cache_seqlens,
                            indices,    sched_meta, num_splits, num_sm_parts, softmax_scale, batch,
                            s_q,        h_q,     topk,       o,           lse};
+  if (int rc = smla::check_decode_call(c)) return rc;
+  if (batch == 0) return SMLA_OK;
+  if (!workspace || !aligned(workspace, 256)) return SMLA_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes < smla::workspace_layout(batch, s_q, h_q, num_sm_parts).total) return SMLA_ERR_INVALID_ARGUMENT;
+  if (int rc = smla::ensure_decode_kernels()) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return smla::launch_decode(c, ws, reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream));
+}
+
+int smla_get_mla_metadata_dense(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int causal,
+                                int num_sm_parts, int32_t* sched_meta, int32_t* num_splits, int32_t* tile_prefix,
+                                void* stream) {
+  if (batch < 0 || s_q < 1 || num_sm_parts < 1 || (causal != 0 && causal != 1) || !sched_meta || !num_splits ||
+      !tile_prefix || (batch > 0 && !cache_seqlens))
+    return SMLA_ERR_INVALID_ARGUMENT;
+  if (!valid_h_q(h_q)) return SMLA_ERR_UNSUPPORTED;
+  if (!aligned(sched_meta, 16)) return SMLA_ERR_INVALID_ARGUMENT;
+  if ((int64_t)batch * s_q > (1 << 28)) return SMLA_ERR_INVALID_ARGUMENT;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(1024);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  if (const cudaError_t e = cudaLaunchKernelEx(&cfg, smla::sched_meta_dense_kernel, cache_seqlens, batch, s_q, causal,
+                                               num_sm_parts, sched_meta, num_splits, tile_prefix);
+      e != cudaSuccess)
+    return smla::cuda_failure(e);
+  return SMLA_OK;
+}
+
+int smla_flash_mla_dense_with_kvcache(const void* q, const uint8_t* kvcache, int kv_format, int64_t num_blocks,
+                                      const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                                      const int32_t* sched_meta, const int32_t* num_splits,
+                                      const int32_t* tile_prefix, int num_sm_parts, float softmax_scale, int causal,
+                                      int batch, int s_q, int h_q, void* o, float* lse, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (kv_format != SMLA_KV_FP8 && kv_format != SMLA_KV_BF16) return SMLA_ERR_INVALID_ARGUMENT;
+  smla::DecodeCall c{q,          kvcache, num_blocks, block_table, max_blocks, cache_seqlens,
+                     nullptr,    sched_meta, num_splits, num_sm_parts, softmax_scale, batch,
+                     s_q,        h_q,     1,          o,           lse};
+  c.tile_prefix = tile_prefix;
+  c.kv_mode = kv_format == SMLA_KV_BF16 ? smla::kDenseBf16 : smla::kDenseFp8;
+  c.causal = causal;
   if (int rc = smla::check_decode_call(c)) return rc;
   if (batch == 0) return SMLA_OK;
   if (!workspace || !aligned(workspace, 256)) return SMLA_ERR_INVALID_ARGUMENT;

@@ -214,6 +214,17 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
                : "memory");
 }
 
+// Store `sel ? a : b` at addr: two predicated stores (each lane executes one)
+// instead of selecting 4 registers of data.
+__device__ __forceinline__ void st_shared_v4_sel(uint32_t addr, bool sel, const uint4& a, const uint4& b) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+      "@p st.shared.v4.u32 [%0], {%2, %3, %4, %5};\n\t"
+      "@!p st.shared.v4.u32 [%0], {%6, %7, %8, %9};\n\t}" ::"r"(addr),
+      "r"((uint32_t)sel), "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+      : "memory");
+}
+
 __device__ __forceinline__ void st_shared_u8(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.u8 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
@@ -239,12 +250,27 @@ __device__ __forceinline__ uint32_t nibbles_to_bits(uint64_t x) {
 
 // Walks a part's (request, tile) range one tile at a time, without any
 // division in the loop.
+// Tiles of request r: the fixed count n_tiles, or (dense decode) the
+// difference of the tile prefix, at least 1 (a table that says otherwise is
+// not from the metadata kernel; clamping keeps every walk finite).
+__device__ __forceinline__ int tiles_of(const SplitKVParams& p, int r) {
+  if (p.tile_prefix == nullptr) return p.n_tiles;
+  const int n = __ldg(p.tile_prefix + r + 1) - __ldg(p.tile_prefix + r);
+  return n > 0 ? n : 1;
+}
+
+// Tiles before request r in the part's (request, tile) order.
+__device__ __forceinline__ int64_t tile_start(const SplitKVParams& p, int r) {
+  return p.tile_prefix == nullptr ? (int64_t)r * p.n_tiles : (int64_t)__ldg(p.tile_prefix + r);
+}
+
 struct Cursor {
-  int r, t;
-  __device__ __forceinline__ void advance(int n) {
+  int r, t, n;   // request, tile within it, tiles of the request
+  __device__ __forceinline__ void advance(const SplitKVParams& p) {
     if (++t == n) {
       t = 0;
       ++r;
+      if (p.tile_prefix != nullptr && r < p.num_requests) n = tiles_of(p, r);
     }
   }
 };
@@ -252,12 +278,13 @@ struct Cursor {
 // The same walk that also tracks the batch entry b = r / s_q of the request
 // (b and q = r % s_q advance with r, so the loop needs no division).
 struct BatchCursor {
-  int r, t, b, q;
-  __device__ __forceinline__ void advance(int n, int s_q) {
+  int r, t, n, b, q;
+  __device__ __forceinline__ void advance(const SplitKVParams& p) {
     if (++t == n) {
       t = 0;
       ++r;
-      if (++q == s_q) {
+      if (p.tile_prefix != nullptr && r < p.num_requests) n = tiles_of(p, r);
+      if (++q == p.s_q) {
         q = 0;
         ++b;
       }
@@ -267,8 +294,12 @@ struct BatchCursor {
 
 }  // namespace
 
-template <bool kPair>
+template <bool kPair, int kMode>
 __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const SplitKVParams p) {
+  constexpr bool kDense = kMode != kSparseFp8;
+  constexpr bool kBf16 = kMode == kDenseBf16;
+  constexpr int kRowBytes = kBf16 ? 1152 : 656;     // one cache row
+  constexpr int kRopeOff = kBf16 ? 1024 : 528;      // byte offset of its 64 bf16 RoPE values
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Tail* tail = reinterpret_cast<Tail*>(smem + kOffTail);
@@ -313,19 +344,22 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
   // Metadata comes from the caller: check it against this call's shapes so a
   // mismatched table cannot send reads or writes out of bounds.
   bool empty = m1.y != 0;
+  int n0 = 1;   // tiles of the part's first request
   if (!empty) {
-    const bool ok = m0.x >= 0 && m0.x < p.num_requests && m0.y >= 0 && m0.y < p.n_tiles && m0.z >= m0.x &&
-                    m0.z <= p.num_requests && m0.w >= 0 && m0.w < p.n_tiles &&
-                    (m0.z > m0.x || m0.w > m0.y) && (m0.z < p.num_requests || m0.w == 0);
+    const int R = p.num_requests;
+    bool ok = m0.x >= 0 && m0.x < R && m0.y >= 0 && m0.z >= m0.x && m0.z <= R && m0.w >= 0;
+    if (ok) {
+      n0 = tiles_of(p, m0.x);
+      ok = m0.y < n0 && (m0.z < R ? m0.w < tiles_of(p, m0.z) : m0.w == 0) && (m0.z > m0.x || m0.w > m0.y);
+    }
     if (!ok) {
       if (tid == 0) report_status(p.status, kStatusBadSchedule);
       empty = true;
     }
   }
-  const int n = p.n_tiles;
-  const int64_t g0 = empty ? 0 : (int64_t)m0.x * n + m0.y;
-  const int64_t g1 = empty ? 0 : (int64_t)m0.z * n + m0.w;
-  const int64_t ntile = g1 - g0;
+  const int64_t g0 = empty ? 0 : tile_start(p, m0.x) + m0.y;
+  const int64_t g1 = empty ? 0 : tile_start(p, m0.z) + m0.w;
+  const int64_t ntile = g1 > g0 ? g1 - g0 : 0;
 
   if (warp >= 4 && warp < 4 + kProducerWarps) {
     // ======================= producers =====================================
@@ -351,20 +385,24 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     const int c_first = 2 * (lane & 3) + swap;
     const int c_second = 2 * (lane & 3) + 1 - swap;
     // tiles t+3 (indices), t+2 (block table), t (fill)
-    BatchCursor ca{m0.x, m0.y, m0.x / p.s_q, m0.x % p.s_q}, cb = ca;
-    Cursor cf{m0.x, m0.y};
+    BatchCursor ca{m0.x, m0.y, n0, m0.x / p.s_q, m0.x % p.s_q}, cb = ca;
+    Cursor cf{m0.x, m0.y, n0};
 
     int idx = -1, sl = 0;        // index and request length of lane k's slot (lanes 0..kRPW-1)
+    int sl_hidden = 0;           // dense causal decode: the request's last positions this token cannot see
     int phys = -1, off = 0;      // its cache block (-1: skip) and row within the block
     bool looked_up = false;      // lane k's slot is valid and its block-table entry was read
     int row_c = -1;              // cache row of lane k's slot in the tile being dequantised
     uint4 lat[kRPW], rp[kRPW / 4];
+    uint4 lat2[kBf16 ? kRPW : 1];  // BF16 rows: the second 16 bytes of each lane's 32
     float sc[kRPW];
 #pragma unroll
     for (int k = 0; k < kRPW; ++k) {
       lat[k] = make_uint4(0u, 0u, 0u, 0u);
       sc[k] = 0.f;
     }
+#pragma unroll
+    for (int k = 0; k < (kBf16 ? kRPW : 1); ++k) lat2[k] = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int i = 0; i < kRPW / 4; ++i) rp[i] = make_uint4(0u, 0u, 0u, 0u);
 
@@ -396,19 +434,22 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
             const __nv_bfloat16* qrow = p.q + ((size_t)cf.r * p.h_q + (size_t)kHeads * hg + (qlive ? qh : 0)) * 576;
             const uint32_t qaddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + kQCol;
             const int c0 = (pw < 4) ? 0 : 5, c1 = (pw < 4) ? 5 : 9;
+            // each chunk in two halves of 8 columns (the two 16-thread halves of
+            // the warp write 16 columns apart), to keep few registers live
 #pragma unroll 1
-            for (int c = c0; c < c1; ++c) {
-              uint32_t v[16];
+            for (int h = 2 * c0; h < 2 * c1; ++h) {
+              const int c = h >> 1, u0 = 2 * (h & 1);
+              uint32_t v[8];
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
+              for (int u = 0; u < 2; ++u) {
                 uint4 x = make_uint4(0u, 0u, 0u, 0u);
-                ldg_v4_if(x, qrow + 64 * c + 32 * (lane >> 4) + 8 * u, qlive);
+                ldg_v4_if(x, qrow + 64 * c + 32 * (lane >> 4) + 8 * (u0 + u), qlive);
                 v[4 * u] = x.x;
                 v[4 * u + 1] = x.y;
                 v[4 * u + 2] = x.z;
                 v[4 * u + 3] = x.w;
               }
-              tmem_st16x2_16(qaddr + 32 * c, v);
+              tmem_st16x2_8<16>(qaddr + 32 * c + 4 * u0, v);
             }
           }
           tmem_wait_st();
@@ -422,17 +463,23 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         }
         const uint32_t vbits = __ballot_sync(0xffffffffu, row_c >= 0) & ((1u << kRPW) - 1u);
         // A skipped slot's registers were zeroed and its loads predicated
-        // off, so dequantising it unconditionally stores a zero row.  Lanes
-        // that store their upper half first swap the two 8-byte halves of
-        // the input instead of the two 16-byte halves of the output.
+        // off, so dequantising (or copying) it unconditionally stores a zero
+        // row.  FP8 rows: lanes that store their upper half first swap the
+        // two 8-byte halves of the input instead of the two 16-byte halves of
+        // the output.  BF16 rows are stored as they are.
 #pragma unroll
         for (int k = 0; k < kRPW; ++k) {
           const int row = rb + k;
-          const uint4 in = swap ? make_uint4(lat[k].z, lat[k].w, lat[k].x, lat[k].y) : lat[k];
-          uint4 first, second;
-          dequant16(in, sc[k], first, second);
-          st_shared_v4(aK + kb * kAtom + swz(row, c_first), first);
-          st_shared_v4(aK + kb * kAtom + swz(row, c_second), second);
+          if constexpr (kBf16) {
+            st_shared_v4_sel(aK + kb * kAtom + swz(row, c_first), swap, lat2[k], lat[k]);
+            st_shared_v4_sel(aK + kb * kAtom + swz(row, c_second), swap, lat[k], lat2[k]);
+          } else {
+            const uint4 in = swap ? make_uint4(lat[k].z, lat[k].w, lat[k].x, lat[k].y) : lat[k];
+            uint4 first, second;
+            dequant16(in, sc[k], first, second);
+            st_shared_v4(aK + kb * kAtom + swz(row, c_first), first);
+            st_shared_v4(aK + kb * kAtom + swz(row, c_second), second);
+          }
         }
 #pragma unroll
         for (int i = 0; i < kRPW / 4; ++i) st_shared_v4(aK + 8 * kAtom + swz(rb + 4 * i + (lane >> 3), lane & 7), rp[i]);
@@ -443,7 +490,7 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
           st_shared_u8(va, nib);
           if (kPair) st_cluster_u8(mapa_shared(va, peer), nib);
         }
-        cf.advance(n);
+        cf.advance(p);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tail->kfull[s]);
@@ -472,38 +519,53 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
 #pragma unroll
         for (int k = 0; k < kRPW; ++k) {
           const int rk = __shfl_sync(0xffffffffu, row_c, k);
-          const uint8_t* row = p.kv + (int64_t)max(rk, 0) * 656;
+          const uint8_t* row = p.kv + (int64_t)max(rk, 0) * kRowBytes;
           lat[k] = make_uint4(0u, 0u, 0u, 0u);
-          sc[k] = 0.f;
-          ldg_v4_evict_first_if(lat[k], row + 16 * lane, rk >= 0, pol);
-          ldg_f32_evict_first_if(sc[k], row + 512 + 4 * (lane >> 3), rk >= 0, pol);
+          if constexpr (kBf16) {
+            // lane l: latent values [16 l, 16 l + 16) = bytes [32 l, 32 l + 32)
+            lat2[k] = make_uint4(0u, 0u, 0u, 0u);
+            ldg_v4_evict_first_if(lat[k], row + 32 * lane, rk >= 0, pol);
+            ldg_v4_evict_first_if(lat2[k], row + 32 * lane + 16, rk >= 0, pol);
+          } else {
+            sc[k] = 0.f;
+            ldg_v4_evict_first_if(lat[k], row + 16 * lane, rk >= 0, pol);
+            ldg_f32_evict_first_if(sc[k], row + 512 + 4 * (lane >> 3), rk >= 0, pol);
+          }
         }
 #pragma unroll
         for (int i = 0; i < kRPW / 4; ++i) {
           const int rk = __shfl_sync(0xffffffffu, row_c, 4 * i + (lane >> 3));
           rp[i] = make_uint4(0u, 0u, 0u, 0u);
-          ldg_v4_evict_first_if(rp[i], p.kv + (int64_t)max(rk, 0) * 656 + 528 + 16 * (lane & 7), rk >= 0, pol);
+          ldg_v4_evict_first_if(rp[i], p.kv + (int64_t)max(rk, 0) * kRowBytes + kRopeOff + 16 * (lane & 7), rk >= 0,
+                                pol);
         }
       }
       // ---- block-table entry of tile R+2 -----------------------------------
       if (R + 2 >= 0 && R + 2 < ntile) {
-        const bool valid = lane < kRPW && idx >= 0 && idx < sl;
+        const bool valid = lane < kRPW && idx >= 0 && idx + sl_hidden < sl;
         const int blk = idx >> 6;
         if (valid && blk >= p.max_blocks) report_status(p.status, kStatusBadBlockTable);
         off = idx & 63;
         phys = -1;
         looked_up = valid && blk < p.max_blocks;
         ldg_s32_if(phys, p.block_table + (size_t)cb.b * p.max_blocks + blk, looked_up);
-        cb.advance(n, p.s_q);
+        cb.advance(p);
       }
       // ---- index and request length of tile R+3 ---------------------------
       if (R + 3 < ntile) {
         const int slot = ca.t * kRows + rb + lane;
         idx = -1;
         sl = 0;
-        ldg_s32_if(idx, p.indices + (size_t)ca.r * p.topk + slot, lane < kRPW && slot < p.topk);
+        if constexpr (kDense) {
+          // every position of the request, in order; the causal mask hides
+          // the last s_q - 1 - t of them from token t
+          if (lane < kRPW) idx = slot;
+          sl_hidden = p.causal ? p.s_q - 1 - ca.q : 0;
+        } else {
+          ldg_s32_if(idx, p.indices + (size_t)ca.r * p.topk + slot, lane < kRPW && slot < p.topk);
+        }
         ldg_s32_if(sl, p.seqlens + ca.b, lane < kRPW);
-        ca.advance(n, p.s_q);
+        ca.advance(p);
       }
     }
     // Every arrive aimed at this CTA's ring barriers (the peer's multicast
@@ -527,11 +589,11 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     const uint32_t k_lo0 = smem_desc_lo(aK0, 16);     // K-major: leading offset 16 bytes
     const uint32_t d_hi = smem_desc_hi_sw128(1024);
     int req_ord = -1;
-    Cursor cm{m0.x, m0.y};
+    Cursor cm{m0.x, m0.y, n0};
 #pragma unroll 1
-    for (int64_t j = 0; j < ntile; ++j, cm.advance(n)) {
+    for (int64_t j = 0; j < ntile; ++j, cm.advance(p)) {
       const bool t_first = (j == 0) || (cm.t == 0);
-      const bool t_last = (j == ntile - 1) || (cm.t == n - 1);
+      const bool t_last = (j == ntile - 1) || (cm.t == cm.n - 1);
       const int s = (int)(j & 1);
       if (t_first) {
         ++req_ord;
@@ -571,13 +633,13 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     int req_ord = -1;
     int slot = 0, nsplit = 1;
     bool req_ok = true;
-    Cursor cx{m0.x, m0.y};
+    Cursor cx{m0.x, m0.y, n0};
 #pragma unroll 1
-    for (int64_t j = 0; j < ntile; ++j, cx.advance(n)) {
+    for (int64_t j = 0; j < ntile; ++j, cx.advance(p)) {
       struct {
         int r;
         bool first, last;
-      } tp{cx.r, (j == 0) || (cx.t == 0), (j == ntile - 1) || (cx.t == n - 1)};
+      } tp{cx.r, (j == 0) || (cx.t == 0), (j == ntile - 1) || (cx.t == cx.n - 1)};
       const int s = (int)(j & 1);
       const uint32_t ph = (uint32_t)((j >> 1) & 1);
       if (tp.first) {
@@ -722,8 +784,18 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
 int splitkv_smem_bytes() { return kSmemBytes; }
 
 // Host launcher shared by the entry points: picks the single-CTA or the
-// two-CTA cluster form and chains the launch to the previous kernel of the
-// stream with programmatic dependent launch.
+// two-CTA cluster form and the key source, and chains the launch to the
+// previous kernel of the stream with programmatic dependent launch.
+template <bool kPair>
+static cudaError_t launch_form(const cudaLaunchConfig_t& cfg, const SplitKVParams& p) {
+  switch (p.kv_mode) {
+    case kSparseFp8: return cudaLaunchKernelEx(&cfg, splitkv_mla_kernel<kPair, kSparseFp8>, p);
+    case kDenseFp8: return cudaLaunchKernelEx(&cfg, splitkv_mla_kernel<kPair, kDenseFp8>, p);
+    case kDenseBf16: return cudaLaunchKernelEx(&cfg, splitkv_mla_kernel<kPair, kDenseBf16>, p);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_splitkv(const SplitKVParams& p, cudaStream_t stream) {
   const bool pair = p.h_q > kHeads;
   cudaLaunchAttribute attrs[2];
@@ -742,15 +814,22 @@ cudaError_t launch_splitkv(const SplitKVParams& p, cudaStream_t stream) {
   cfg.stream = stream;
   cfg.attrs = attrs;
   cfg.numAttrs = pair ? 2 : 1;
-  if (pair) return cudaLaunchKernelEx(&cfg, splitkv_mla_kernel<true>, p);
-  return cudaLaunchKernelEx(&cfg, splitkv_mla_kernel<false>, p);
+  return pair ? launch_form<true>(cfg, p) : launch_form<false>(cfg, p);
+}
+
+template <bool kPair, int kMode>
+static cudaError_t set_smem() {
+  return cudaFuncSetAttribute(splitkv_mla_kernel<kPair, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kSmemBytes);
 }
 
 cudaError_t configure_splitkv() {
-  cudaError_t e =
-      cudaFuncSetAttribute(splitkv_mla_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(splitkv_mla_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  const cudaError_t e[6] = {set_smem<true, kSparseFp8>(), set_smem<false, kSparseFp8>(),
+                            set_smem<true, kDenseFp8>(),  set_smem<false, kDenseFp8>(),
+                            set_smem<true, kDenseBf16>(), set_smem<false, kDenseBf16>()};
+  for (cudaError_t x : e)
+    if (x != cudaSuccess) return x;
+  return cudaSuccess;
 }
 
 }  // namespace smla

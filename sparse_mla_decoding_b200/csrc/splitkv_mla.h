@@ -11,17 +11,27 @@
 
 namespace smla {
 
+// What the split kernel reads for a request's keys.
+enum KvMode : int {
+  kSparseFp8 = 0,   // the indices tensor names the tokens; 656-byte FP8 rows
+  kDenseFp8 = 1,    // every visible token (indices made in the kernel); 656-byte FP8 rows
+  kDenseBf16 = 2,   // every visible token; 1152-byte BF16 rows (576 bf16 values)
+};
+
 struct SplitKVParams {
   const __nv_bfloat16* q;       // [R][h_q][576], R = batch * s_q
-  const uint8_t* kv;            // [num_blocks][64][656]
+  const uint8_t* kv;            // [num_blocks][64][row bytes]
   int64_t num_blocks;
   const int32_t* block_table;   // [batch][max_blocks]
   int max_blocks;
   const int32_t* seqlens;       // [batch]
-  const int32_t* indices;       // [R][topk]
+  const int32_t* indices;       // [R][topk] (sparse mode)
+  const int32_t* tile_prefix;   // [R + 1] tiles before each request (dense modes), or nullptr
+  int kv_mode;                  // KvMode
+  int causal;                   // dense modes: token t of s_q sees seqlen - (s_q - 1 - t) positions
   const int32_t* sched_meta;    // [num_parts][8]
   const int32_t* num_splits;    // [R + 1]
-  int s_q, h_q, topk, n_tiles, num_parts;
+  int s_q, h_q, topk, n_tiles, num_parts;   // n_tiles: tiles per request when tile_prefix is nullptr
   int num_requests;             // R = batch * s_q
   int max_splits;               // split slots the workspace holds (R + num_parts)
   float scale_log2;             // softmax_scale * log2(e)
@@ -64,6 +74,10 @@ struct DecodeCall {
   int batch, s_q, h_q, topk;
   void* o;
   float* lse;
+  // dense decode (left at their defaults by the sparse entry points)
+  const int32_t* tile_prefix = nullptr;
+  int kv_mode = kSparseFp8;
+  int causal = 0;
 };
 
 // Records a failing CUDA runtime result for smla_last_cuda_error (one slot
