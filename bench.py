@@ -301,13 +301,12 @@ def make_device_copy(w, device, values="host"):
 # Reported only while they still match; the capture commands are in profiles/.
 NCU_TRAFFIC = {
     "decode_h128_b64_topk2048": {
-        "bytes": 107_550_720 + 5_125_376,
-        "srchash": "dc378b35c53c2791723f2adcf6c66e4763ab184b230c13c99d0fd6b47e36a918"},
+        "bytes": 107_526_400 + 4_323_840,
+        "srchash": "0f562194fe5cd146591b491bfb0e8e75170d243132f99d4d1c2a69077c0e1e05"},
     "decode_h64_b128_sq2_topk2048": {
-        "bytes": 395_680_768 + 5_133_056,
-        "srchash": "dc378b35c53c2791723f2adcf6c66e4763ab184b230c13c99d0fd6b47e36a918"},
+        "bytes": 395_768_320 + 4_065_536,
+        "srchash": "0f562194fe5cd146591b491bfb0e8e75170d243132f99d4d1c2a69077c0e1e05"},
 }
-
 
 def split_kernel_hash():
     """Hash of the files the split kernel is compiled from (and of the build flags)."""
@@ -482,6 +481,91 @@ def decode_record(w, n_copies, values, mode, l2_note, args, device, rank, world,
     return rec
 
 
+# Dense decode shapes (every cached token attended; the pages give no shapes
+# for it): 64 requests of 8192 tokens, 128 heads, one new token, FP8 or BF16
+# cache rows.  Each step gathers 344 MB (FP8) or 604 MB (BF16) of rows, both
+# larger than the 126 MB L2, from one copy.
+DENSE_RECORDS = (("dense_fp8_h128_b64_s8192", 0), ("dense_bf16_h128_b64_s8192", 1))
+
+
+def dense_record(name, kv_format, args, device, rank, world, peaks):
+    """Dense decode (metadata + split kernel + combine) on one paged cache."""
+    import torch
+    import sparse_mla_decoding_b200 as smla
+    from sparse_mla_decoding_b200 import workloads as W
+    w = W.Workload(name, batch=64, s_q=1, h_q=128, topk=1, seed=rank_seed(W.DECODE_H128, rank, 5 + kv_format),
+                   seqlens=(8192,) * 64)
+    stream = torch.cuda.current_stream(device)
+    lay = W.layout(w)
+    rows = lay.num_blocks * W.BLOCK
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(w.seed) * 131 + 7)
+    if kv_format == 0:
+        kv = torch.empty((lay.num_blocks, W.BLOCK, ROW), dtype=torch.uint8, device=device)
+        flat = kv.view(rows, ROW)
+        for start in range(0, rows, 1 << 20):
+            n = min(1 << 20, rows - start)
+            smla.quantize_kv(torch.randn((n, DV), generator=gen, device=device).to(torch.bfloat16),
+                             torch.randn((n, 64), generator=gen, device=device).to(torch.bfloat16), flat[start:start + n])
+        row_bytes = ROW
+    else:
+        kv = torch.randn((lay.num_blocks, W.BLOCK, DQK), generator=gen, device=device).to(torch.bfloat16)
+        row_bytes = 2 * DQK
+    q = torch.from_numpy(W.queries(w).view(np.int16)).to(device).view(torch.bfloat16)
+    bt = torch.from_numpy(lay.block_table).to(device)
+    sl = torch.from_numpy(lay.seqlens.astype(np.int32)).to(device)
+    tokens = float(lay.seqlens.sum()) * w.s_q
+    flops = 2.0 * w.h_q * (DQK + DV) * tokens
+    parts = smla.default_num_sm_parts(w.h_q, device)
+    ws = smla.new_workspace(w.batch, w.s_q, w.h_q, 1, parts, device)
+    outs = (torch.empty((w.batch, w.s_q, w.h_q, DV), dtype=torch.bfloat16, device=device),
+            torch.empty((w.batch, w.s_q, w.h_q), dtype=torch.float32, device=device))
+    meta = smla.get_mla_metadata_dense(sl, w.h_q, s_q=w.s_q, causal=True, num_sm_parts=parts)
+
+    def step(i):
+        sm, ns, tp = smla.get_mla_metadata_dense(sl, w.h_q, s_q=w.s_q, causal=True, num_sm_parts=parts)
+        smla.flash_mla_dense_with_kvcache(q, kv, bt, sl, sm, ns, tp, causal=True, workspace=ws, out=outs)
+
+    def call(i):
+        smla.flash_mla_dense_with_kvcache(q, kv, bt, sl, *meta, causal=True, workspace=ws, out=outs)
+
+    for i in range(args.warmup):
+        step(i)
+    steps = max(args.steps // 2, 8)
+    step_ms = timed(step, steps, stream)
+    call_ms = timed(call, steps, stream)
+    status, raw = smla.get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status word set during the {name} record: {raw:#x}")
+    (step_ms, call_ms), (f_all, b_all) = reduce_over_ranks([step_ms, call_ms], [flops, tokens * row_bytes], device,
+                                                           world)
+    rec = {"value": f_all / (step_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": step_ms, "steps": steps,
+           "gathered_kv_gbs": b_all / (step_ms * 1e-3) / 1e9,
+           "roofline": dict(roofline(peaks, w.h_q, flops, tokens * row_bytes, call_ms) if kv_format == 0 else
+                            _dense_bf16_roofline(peaks, flops, tokens * row_bytes, call_ms),
+                            kernel="splitkv_mla_kernel + combine_kernel (one dense decode call)", kernel_ms=call_ms,
+                            peak_source=peaks["source"] + " (burst)"),
+           "config": {"api": "flash_mla_dense_with_kvcache", "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q,
+                      "seqlen": 8192, "causal": True, "kv_row_bytes": row_bytes,
+                      "cache_values": "seeded torch generator on the GPU",
+                      "l2": f"one copy: {tokens * row_bytes / 1e6:.0f} MB of rows per step > 126 MB L2"}}
+    del kv, ws, q
+    torch.cuda.empty_cache()
+    return rec
+
+
+def _dense_bf16_roofline(peaks, flops, nbytes, ms):
+    """BF16 rows carry 1152 bytes for 2 * 128 * 1088 flop: compare both roofs, report the binding one."""
+    intensity = flops / nbytes
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if intensity >= ridge:
+        a = flops / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": a, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": a / peaks["bf16_tflops"]}
+    a = nbytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": a, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": a / peaks["hbm_gbs"]}
+
+
 def sparse_fwd_record(args, device, rank, world, peaks):
     """flash_mla_sparse_fwd on the prefill-shaped workload: 4096 query tokens over one flat FP8 cache."""
     import torch
@@ -653,6 +737,8 @@ def run_ours(args, w, rank, world, local_rank):
                 if name != w.name:
                     decode_record(W.BY_NAME[name], n_copies, values, mode, note, args, device, rank, world, peaks)
             sparse_fwd_record(args, device, rank, world, peaks)
+            for name, fmt in DENSE_RECORDS:
+                dense_record(name, fmt, args, device, rank, world, peaks)
         return
 
     tflops = tot_flops / (ms_total * 1e-3) / 1e12
@@ -697,6 +783,8 @@ def run_ours(args, w, rank, world, local_rank):
                 continue
             extra[name] = decode_record(W.BY_NAME[name], n_copies, values, mode, note, args, device, rank, world, peaks)
         extra["sparse_fwd_prefill_shaped_h128_sq4096_topk2048"] = sparse_fwd_record(args, device, rank, world, peaks)
+        for name, fmt in DENSE_RECORDS:
+            extra[name] = dense_record(name, fmt, args, device, rank, world, peaks)
         line["workloads"] = extra
     print(json.dumps(line), flush=True)
 
