@@ -86,10 +86,23 @@ const char* smla_last_cuda_error_string(void);
 /*
  * Default number of scheduler parts for h_q heads on `device`: one part per
  * CTA group that can be resident at once (the SM count for h_q <= 64; half of
- * it for h_q = 128, where a part is a pair of CTAs that own 64 heads each).
+ * it for h_q = 128, where a part is two CTAs that own 64 heads each).
  * Returns a value >= 1, or -1 if the device cannot be queried.
  */
 int smla_default_num_sm_parts(int h_q, int device);
+
+/*
+ * How the two 64-head CTAs of a 128-head part share a tile ("FlashMLA
+ * 注意力内核源码走读…", section 计算环节一, describes the shared form).
+ *   enable = 0 (default): independent CTAs; each gathers and dequantises all
+ *                64 rows of a tile (the second read of a row mostly hits L2).
+ *   enable = 1: a two-CTA cluster; each CTA dequantises half of the rows and
+ *                copies them into its peer's shared memory.
+ * Both forms give bitwise identical results; on B200 the independent form
+ * measured faster.  The setting is process-wide, takes effect at the next
+ * decode call, and returns the previous setting.
+ */
+int smla_set_head_pair_form(int enable);
 
 /*
  * Bytes of caller-provided device workspace that smla_flash_mla_with_kvcache
@@ -124,12 +137,12 @@ int smla_get_mla_metadata(const int32_t* cache_seqlens, int batch, int s_q, int 
 
 /*
  * Sparse MLA decode ("FlashMLA 注意力内核源码走读…", sections 解码阶段调用示例,
- * 数据加载, 合并与性能账本).  Launches the split-KV kernel (one CTA, or a
- * pair of CTAs for 128 heads, per scheduler part, each walking its part's
- * (request, tile) ranges from sched_meta) and, chained to it with
- * Programmatic Dependent Launch, the LSE combine kernel for requests that
- * were split.  Output is bitwise reproducible run to run (static schedule,
- * no floating-point atomics).
+ * 数据加载, 合并与性能账本).  Launches the split-KV kernel (one CTA per
+ * scheduler part and 64-head group, see smla_set_head_pair_form, each
+ * walking its part's (request, tile) ranges from sched_meta) and, chained to
+ * it with Programmatic Dependent Launch, the LSE combine kernel for requests
+ * that were split.  Output is bitwise reproducible run to run (static
+ * schedule, no floating-point atomics).
  *   q             : device bf16 [batch][s_q][h_q][576]
  *   kvcache       : device uint8 [num_blocks][64][656] (16-byte aligned);
  *                   num_blocks <= 33554431 (rows are numbered with 32 bits)

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
             L.smla_last_cuda_error.restype = i32
             L.smla_last_cuda_error_string.argtypes = []
             L.smla_last_cuda_error_string.restype = ctypes.c_char_p
+            L.smla_set_head_pair_form.argtypes = [i32]
+            L.smla_set_head_pair_form.restype = i32
             L.smla_default_num_sm_parts.argtypes = [i32, i32]
             L.smla_default_num_sm_parts.restype = i32
             L.smla_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
@@ -104,6 +106,13 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 def _require(cond: bool, msg: str) -> None:
     if not cond:
         raise ValueError(msg)
+
+
+def set_head_pair_form(enable: bool) -> bool:
+    """Run 128-head decodes as two-CTA clusters that share dequantised tiles
+    (True) or as independent CTAs (False, the default); returns the previous
+    setting.  Process-wide; results are bitwise identical either way."""
+    return bool(lib().smla_set_head_pair_form(1 if enable else 0))
 
 
 def default_num_sm_parts(h_q: int, device: Optional[torch.device] = None) -> int:

@@ -12,10 +12,11 @@
 // anywhere) gives o = 0, lse = -inf.  Requests with one split were finished
 // by the split kernel and are skipped.
 //
-// The merge is bound by reading the fp32 partials, so the layout is chosen for
-// memory-level parallelism: one warp per (request, head), lane l owning the 16
-// output columns [16 l, 16 l + 16) (four 16-byte loads per split), with the
-// loads of two splits in flight before either is used.
+// The merge is bound by the latency of reading the fp32 partials, so the
+// layout is chosen for memory-level parallelism: one warp per (request, head),
+// lane l owning the 16 output columns [16 l, 16 l + 16) (four 16-byte loads
+// per split), with the rows of the first two splits loaded before the lse
+// reductions, so their round trip overlaps the lse loads'.
 #include <cuda_bf16.h>
 
 #include <cstdint>
@@ -43,6 +44,14 @@ __global__ void __launch_bounds__(32 * kCombineHeadsPerCta) combine_kernel(const
   if (h >= h_q || ns <= 1 || s0 < 0 || s0 + ns > max_splits) return;
 
   const float* lse_s = lse_accum + (size_t)s0 * h_q + h;   // split s at lse_s[s * h_q]
+  const size_t split_stride = (size_t)h_q * 512;
+  const float* base = o_accum + ((size_t)s0 * h_q + h) * 512 + 16 * lane;
+  float4 va[4], vb[4];   // splits s and s + 1 of the loop below, the first pair loaded now
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    va[i] = reinterpret_cast<const float4*>(base)[i];
+    vb[i] = reinterpret_cast<const float4*>(base + split_stride)[i];
+  }
   float m = -INFINITY;
   for (int s = lane; s < ns; s += 32) m = fmaxf(m, lse_s[(size_t)s * h_q]);
 #pragma unroll
@@ -65,17 +74,16 @@ __global__ void __launch_bounds__(32 * kCombineHeadsPerCta) combine_kernel(const
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  const size_t split_stride = (size_t)h_q * 512;
-  const float* base = o_accum + ((size_t)s0 * h_q + h) * 512 + 16 * lane;
   for (int s = 0; s < ns; s += 2) {
     const bool two = s + 1 < ns;
-    const float4* a = reinterpret_cast<const float4*>(base + (size_t)s * split_stride);
-    const float4* b = reinterpret_cast<const float4*>(base + (size_t)(two ? s + 1 : s) * split_stride);
-    float4 va[4], vb[4];
+    if (s > 0) {
+      const float4* a = reinterpret_cast<const float4*>(base + (size_t)s * split_stride);
+      const float4* b = reinterpret_cast<const float4*>(base + (size_t)(two ? s + 1 : s) * split_stride);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      va[i] = a[i];
-      vb[i] = b[i];
+      for (int i = 0; i < 4; ++i) {
+        va[i] = a[i];
+        vb[i] = b[i];
+      }
     }
     const float wa = exp2f((lse_s[(size_t)s * h_q] - lse_r) * kLog2e);
     const float wb = two ? exp2f((lse_s[(size_t)(s + 1) * h_q] - lse_r) * kLog2e) : 0.f;

@@ -314,26 +314,22 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return pol;
 }
 
+// Unconditional 16- and 4-byte loads with that policy (callers point a
+// skipped row at a zero row rather than predicating the load).
+__device__ __forceinline__ void ldg_v4_evict_first(uint4& v, const void* p, uint64_t pol) {
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+}
+
+__device__ __forceinline__ void ldg_f32_evict_first(float& v, const void* p, uint64_t pol) {
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(v) : "l"(p), "l"(pol));
+}
+
 // Predicated loads: when `pred` is false the destination keeps its previous
 // value and no instruction reads the (pending) load result, so a load can be
 // issued long before its use even when it is conditional.  (A plain
 // `v = 0; if (pred) v = load;` becomes a select that waits for the load.)
-__device__ __forceinline__ void ldg_v4_evict_first_if(uint4& v, const void* p, bool pred, uint64_t pol) {
-  asm volatile(
-      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %5, 0;\n\t"
-      "@q ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %6;\n\t}"
-      : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)
-      : "l"(p), "r"((uint32_t)pred), "l"(pol));
-}
-
-__device__ __forceinline__ void ldg_f32_evict_first_if(float& v, const void* p, bool pred, uint64_t pol) {
-  asm volatile(
-      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t"
-      "@q ld.global.nc.L1::no_allocate.L2::cache_hint.f32 %0, [%1], %3;\n\t}"
-      : "+f"(v)
-      : "l"(p), "r"((uint32_t)pred), "l"(pol));
-}
-
 __device__ __forceinline__ void ldg_v4_if(uint4& v, const void* p, bool pred) {
   asm volatile(
       "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %5, 0;\n\t"
@@ -348,6 +344,14 @@ __device__ __forceinline__ void ldg_s32_if(int& v, const void* p, bool pred) {
       "@q ld.global.nc.s32 %0, [%1];\n\t}"
       : "+r"(v)
       : "l"(p), "r"((uint32_t)pred));
+}
+
+// Brings the cache line holding `p` into L2 ahead of its load (no register
+// result, nothing waits for it).
+__device__ __forceinline__ void prefetch_l2_if(const void* p, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+      "@q prefetch.global.L2 [%0];\n\t}" ::"l"(p), "r"((uint32_t)pred));
 }
 
 // PDL (programmatic dependent launch) controls.

@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -46,6 +47,7 @@ cudaLaunchAttribute pdl_attribute() {
 }
 
 std::mutex g_setup_mutex;
+std::atomic<int> g_head_pair_form{0};
 void* g_configured_ctx[kMaxDevices] = {nullptr};
 
 }  // namespace
@@ -76,6 +78,8 @@ thread_local int g_last_cuda_error = 0;
 }  // namespace
 
 int g_last_cuda_error_value() { return g_last_cuda_error; }
+
+int head_pair_form() { return g_head_pair_form.load(std::memory_order_relaxed); }
 
 int cuda_failure(cudaError_t e) {
   g_last_cuda_error = (int)e;
@@ -147,6 +151,7 @@ int launch_decode(const DecodeCall& c, uint8_t* scratch, uint32_t* status, cudaS
   p.indices = c.indices;
   p.tile_prefix = c.tile_prefix;
   p.kv_mode = c.kv_mode;
+  p.cta_pairs = head_pair_form();
   p.causal = c.causal;
   p.sched_meta = c.sched_meta;
   p.num_splits = c.num_splits;
@@ -197,7 +202,9 @@ const char* smla_status_string(int status) {
   }
 }
 
-int smla_version(void) { return 101; }
+int smla_version(void) { return 102; }
+
+int smla_set_head_pair_form(int enable) { return g_head_pair_form.exchange(enable != 0 ? 1 : 0); }
 
 int smla_last_cuda_error(void) { return smla::g_last_cuda_error_value(); }
 

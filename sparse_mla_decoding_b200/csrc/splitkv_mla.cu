@@ -20,11 +20,15 @@
 //
 // Design on B200:
 //   * A CTA owns 64 query heads of one request at a time (M = 64 of every
-//     tcgen05.mma).  128 heads run as a two-CTA cluster (one CTA per 64-head
-//     group) that shares the dequantised tiles over distributed shared memory
-//     (each CTA dequantises half of the rows, and the copy engine sends them
-//     to the peer with bulk shared-to-shared copies);
-//     16/32 heads are zero-padded to 64 in a single CTA.
+//     tcgen05.mma); 16/32 heads are zero-padded to 64 in a single CTA.  128
+//     heads run, by default, as two independent CTAs per part (one per
+//     64-head group, grid.y), each gathering and dequantising every row of
+//     a tile; the second CTA's reads of a row mostly hit L2.  The optional
+//     two-CTA cluster form shares the dequantised tiles over distributed
+//     shared memory instead (each CTA dequantises half of the rows, and the
+//     copy engine sends them to the peer with bulk shared-to-shared copies):
+//     it halves the dequantisation per CTA but couples every tile of the two
+//     CTAs, and measured slower on B200.
 //   * Warp roles (416 threads, 13 warps, at most 128 registers a thread: one
 //     SM sub-partition holds 4 of the 13 warps):
 //       warps 0-3   softmax: online softmax over S in TMEM (two threads per
@@ -44,10 +48,11 @@
 //     current ones; PV = P V with P and V in shared memory, issued by the
 //     softmax warpgroup itself right after it has written P (no hand-off to
 //     another warp on the per-tile critical path).
-//   * The producers run a four-stage software pipeline across tiles
-//     (dequantise tile t, row loads of t+1, block table of t+2, indices of
-//     t+3), so the dependent loads index -> block table -> row never stall
-//     a tile and the rows are in flight while the ring slot drains.
+//   * The producers run a five-stage software pipeline across tiles
+//     (dequantise tile t, row loads of t+1, L2 prefetch of the rows of t+2,
+//     block table of t+3, indices of t+4), so the dependent loads index ->
+//     block table -> row never stall a tile, the rows of t+1 are in flight
+//     while the ring slot drains, and they come from L2 rather than DRAM.
 //   * TMEM (512 columns; an M = 64 operand or accumulator uses 16 lanes of
 //     each 32-lane sub-partition): lanes 0-15 hold Q (64 x 576 bf16, two
 //     values a column, columns [0, 288)) and the S double buffer (columns
@@ -117,6 +122,12 @@ struct __align__(16) Tail {
   uint32_t tmem_base;
 };
 static_assert(offsetof(Tail, vmask) % 16 == 0 && offsetof(Tail, kfull) % 8 == 0, "Tail field alignment");
+
+// The source of a skipped slot's row loads: zeros (a __device__ array is
+// zero-initialised when the module loads and nothing writes it), so a
+// skipped slot dequantises to a zero row without predicated loads or
+// register clears.  Sized for the widest row format.
+__device__ __align__(128) uint8_t g_zero_row[1152];
 
 constexpr int kOffK = 0;
 constexpr int kOffP = 2 * kTileBytes;
@@ -190,9 +201,22 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Two round-to-nearest f32 products in one packed instruction (sm_100):
+// (a.x * s, a.y * s), each rounded exactly as a scalar multiply.
+__device__ __forceinline__ float2 fmul2_rn(float2 a, float s) {
+  uint64_t v, sc, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(sc) : "f"(s));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(v), "l"(sc));
+  float2 out;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(out.x), "=f"(out.y) : "l"(r));
+  return out;
+}
+
 // 16 e4m3 values (one 16-byte chunk) -> 16 bf16 = bf16(float(e4m3) * scale):
 // hardware e4m3x2 -> f16x2 converts (exact), f16 -> f32 (exact), a
-// round-to-nearest f32 multiply, then round-to-nearest-even to bf16.
+// round-to-nearest f32 multiply (two per instruction), then
+// round-to-nearest-even to bf16.
 __device__ __forceinline__ void dequant16(const uint4& raw, float scale, uint4& lo, uint4& hi) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
   uint32_t out[8];
@@ -200,10 +224,10 @@ __device__ __forceinline__ void dequant16(const uint4& raw, float scale, uint4& 
   for (int j = 0; j < 4; ++j) {
     __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[j] & 0xFFFFu), __NV_E4M3);
     __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[j] >> 16), __NV_E4M3);
-    float2 f01 = __half22float2(*reinterpret_cast<__half2*>(&h01));
-    float2 f23 = __half22float2(*reinterpret_cast<__half2*>(&h23));
-    out[2 * j] = bf162_bits(__floats2bfloat162_rn(__fmul_rn(f01.x, scale), __fmul_rn(f01.y, scale)));
-    out[2 * j + 1] = bf162_bits(__floats2bfloat162_rn(__fmul_rn(f23.x, scale), __fmul_rn(f23.y, scale)));
+    const float2 p01 = fmul2_rn(__half22float2(*reinterpret_cast<__half2*>(&h01)), scale);
+    const float2 p23 = fmul2_rn(__half22float2(*reinterpret_cast<__half2*>(&h23)), scale);
+    out[2 * j] = bf162_bits(__floats2bfloat162_rn(p01.x, p01.y));
+    out[2 * j + 1] = bf162_bits(__floats2bfloat162_rn(p23.x, p23.y));
   }
   lo = make_uint4(out[0], out[1], out[2], out[3]);
   hi = make_uint4(out[4], out[5], out[6], out[7]);
@@ -339,6 +363,11 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
 
   // The schedule is written by the metadata kernel that precedes us.
   pdl_wait_primary();
+  // Let the combine kernel launch now: its CTAs take whatever room is left
+  // on the SMs (or that finished parts free) and wait in griddepcontrol.wait,
+  // which returns only once this whole grid has completed, so the merge
+  // starts without a launch gap.
+  pdl_launch_dependents();
   const int4 m0 = *reinterpret_cast<const int4*>(p.sched_meta + (size_t)part * 8);
   const int4 m1 = *reinterpret_cast<const int4*>(p.sched_meta + (size_t)part * 8 + 4);
   // Metadata comes from the caller: check it against this call's shapes so a
@@ -365,14 +394,16 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     // ======================= producers =====================================
     // Warp pw owns kRPW consecutive rows of every tile: 8 in the single-CTA
     // form, 4 in the two-CTA form (where a CTA dequantises 32 of the 64 rows
-    // and sends them to its peer).  Tiles are software-pipelined over four
+    // and sends them to its peer).  Tiles are software-pipelined over five
     // stages per iteration, in this order: dequantise tile t, load the rows
-    // of tile t+1, the block-table entries of tile t+2 and the indices of
-    // tile t+3.  Each stage reads what the next one loaded an iteration
-    // earlier, before that register is reloaded, so no load is waited on
-    // early, and the rows of tile t+1 are in flight while the warp waits for
-    // the next ring slot.  The loop body is kept small (one copy of each
-    // stage): the roles share the SM's instruction caches.
+    // of tile t+1, prefetch the rows of tile t+2 into L2, load the
+    // block-table entries of tile t+3 and the indices of tile t+4.  Each
+    // stage reads what the next one produced an iteration earlier, before
+    // that register is reloaded, so no load is waited on early; the rows of
+    // tile t+1 are in flight while the warp waits for the next ring slot,
+    // and the prefetch an iteration earlier has brought them from DRAM into
+    // L2.  The loop body is kept small (one copy of each stage): the roles
+    // share the SM's instruction caches.
     constexpr int kRPW = kPair ? 4 : 8;
     const int pw = warp - 4;
     const uint64_t pol = l2_evict_first_policy();
@@ -384,7 +415,7 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     const int swap = (lane >> 2) & 1;
     const int c_first = 2 * (lane & 3) + swap;
     const int c_second = 2 * (lane & 3) + 1 - swap;
-    // tiles t+3 (indices), t+2 (block table), t (fill)
+    // tiles t+4 (indices), t+3 (block table), t (fill)
     BatchCursor ca{m0.x, m0.y, n0, m0.x / p.s_q, m0.x % p.s_q}, cb = ca;
     Cursor cf{m0.x, m0.y, n0};
 
@@ -392,6 +423,7 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     int sl_hidden = 0;           // dense causal decode: the request's last positions this token cannot see
     int phys = -1, off = 0;      // its cache block (-1: skip) and row within the block
     bool looked_up = false;      // lane k's slot is valid and its block-table entry was read
+    int row_n = -1;              // cache row of lane k's slot in the tile being prefetched
     int row_c = -1;              // cache row of lane k's slot in the tile being dequantised
     uint4 lat[kRPW], rp[kRPW / 4];
     uint4 lat2[kBf16 ? kRPW : 1];  // BF16 rows: the second 16 bytes of each lane's 32
@@ -409,7 +441,7 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     int req_ord = -1;
     bool ok = true;
 #pragma unroll 1
-    for (int64_t R = -3; R < ntile && ok; ++R) {
+    for (int64_t R = -4; R < ntile && ok; ++R) {
       // ---- dequantise and store tile R -------------------------------------
       if (R >= 0) {
         const int64_t j = R;
@@ -462,9 +494,8 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
           break;
         }
         const uint32_t vbits = __ballot_sync(0xffffffffu, row_c >= 0) & ((1u << kRPW) - 1u);
-        // A skipped slot's registers were zeroed and its loads predicated
-        // off, so dequantising (or copying) it unconditionally stores a zero
-        // row.  FP8 rows: lanes that store their upper half first swap the
+        // A skipped slot's registers were loaded from the zero row, so
+        // dequantising (or copying) it unconditionally stores a zero row.  FP8 rows: lanes that store their upper half first swap the
         // two 8-byte halves of the input instead of the two 16-byte halves of
         // the output.  BF16 rows are stored as they are.
 #pragma unroll
@@ -508,40 +539,53 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       }
       // ---- row loads of tile R+1 -------------------------------------------
       if (R + 1 >= 0 && R + 1 < ntile) {
-        // A valid slot whose block-table entry lies outside the cache
-        // (negative or past num_blocks) is skipped and flagged.
-        row_c = -1;
-        if (phys >= 0 && phys < p.num_blocks) row_c = phys * 64 + off;
-        else if (looked_up) report_status(p.status, kStatusBadBlockTable);
+        row_c = row_n;
         // For every row, lane l takes latent bytes [16l, 16l+16) and the scale
         // of its 128-value tile; the RoPE chunks (8 per row) are spread over
-        // the lanes (row 4i + l/8, chunk l%8).
+        // the lanes (row 4i + l/8, chunk l%8).  A skipped slot reads the zero
+        // row instead.
 #pragma unroll
         for (int k = 0; k < kRPW; ++k) {
           const int rk = __shfl_sync(0xffffffffu, row_c, k);
-          const uint8_t* row = p.kv + (int64_t)max(rk, 0) * kRowBytes;
-          lat[k] = make_uint4(0u, 0u, 0u, 0u);
+          const uint8_t* row = rk >= 0 ? p.kv + (int64_t)rk * kRowBytes : g_zero_row;
           if constexpr (kBf16) {
             // lane l: latent values [16 l, 16 l + 16) = bytes [32 l, 32 l + 32)
-            lat2[k] = make_uint4(0u, 0u, 0u, 0u);
-            ldg_v4_evict_first_if(lat[k], row + 32 * lane, rk >= 0, pol);
-            ldg_v4_evict_first_if(lat2[k], row + 32 * lane + 16, rk >= 0, pol);
+            ldg_v4_evict_first(lat[k], row + 32 * lane, pol);
+            ldg_v4_evict_first(lat2[k], row + 32 * lane + 16, pol);
           } else {
-            sc[k] = 0.f;
-            ldg_v4_evict_first_if(lat[k], row + 16 * lane, rk >= 0, pol);
-            ldg_f32_evict_first_if(sc[k], row + 512 + 4 * (lane >> 3), rk >= 0, pol);
+            ldg_v4_evict_first(lat[k], row + 16 * lane, pol);
+            ldg_f32_evict_first(sc[k], row + 512 + 4 * (lane >> 3), pol);
           }
         }
 #pragma unroll
         for (int i = 0; i < kRPW / 4; ++i) {
           const int rk = __shfl_sync(0xffffffffu, row_c, 4 * i + (lane >> 3));
-          rp[i] = make_uint4(0u, 0u, 0u, 0u);
-          ldg_v4_evict_first_if(rp[i], p.kv + (int64_t)max(rk, 0) * kRowBytes + kRopeOff + 16 * (lane & 7), rk >= 0,
-                                pol);
+          const uint8_t* row = rk >= 0 ? p.kv + (int64_t)rk * kRowBytes : g_zero_row;
+          ldg_v4_evict_first(rp[i], row + kRopeOff + 16 * (lane & 7), pol);
         }
       }
-      // ---- block-table entry of tile R+2 -----------------------------------
+      // ---- L2 prefetch of the rows of tile R+2 --------------------------------
       if (R + 2 >= 0 && R + 2 < ntile) {
+        // A valid slot whose block-table entry lies outside the cache
+        // (negative or past num_blocks) is skipped and flagged.
+        row_n = -1;
+        if (phys >= 0 && phys < p.num_blocks) row_n = phys * 64 + off;
+        else if (looked_up) report_status(p.status, kStatusBadBlockTable);
+        // (row, line) pairs over the lanes: each row's 128-byte lines at
+        // offsets 0, 128, ... and its last byte (a row may straddle one more)
+        constexpr int kLines = (kRowBytes + 127) / 128 + 1;
+#pragma unroll 1
+        for (int e0 = 0; e0 < kRPW * kLines; e0 += 32) {
+          const int e = e0 + lane;
+          const int k = min(e / kLines, kRPW - 1);
+          const int rk = __shfl_sync(0xffffffffu, row_n, k);
+          const int li = e - k * kLines;
+          prefetch_l2_if(p.kv + (int64_t)max(rk, 0) * kRowBytes + min(128 * li, kRowBytes - 1),
+                         rk >= 0 && e < kRPW * kLines);
+        }
+      }
+      // ---- block-table entry of tile R+3 -----------------------------------
+      if (R + 3 >= 0 && R + 3 < ntile) {
         const bool valid = lane < kRPW && idx >= 0 && idx + sl_hidden < sl;
         const int blk = idx >> 6;
         if (valid && blk >= p.max_blocks) report_status(p.status, kStatusBadBlockTable);
@@ -551,8 +595,8 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         ldg_s32_if(phys, p.block_table + (size_t)cb.b * p.max_blocks + blk, looked_up);
         cb.advance(p);
       }
-      // ---- index and request length of tile R+3 ---------------------------
-      if (R + 3 < ntile) {
+      // ---- index and request length of tile R+4 ---------------------------
+      if (R + 4 < ntile) {
         const int slot = ca.t * kRows + rb + lane;
         idx = -1;
         sl = 0;
@@ -771,7 +815,6 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
     }
   }
 
-  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (kPair) cluster_sync();
@@ -797,7 +840,7 @@ static cudaError_t launch_form(const cudaLaunchConfig_t& cfg, const SplitKVParam
 }
 
 cudaError_t launch_splitkv(const SplitKVParams& p, cudaStream_t stream) {
-  const bool pair = p.h_q > kHeads;
+  const bool pair = p.h_q > kHeads && p.cta_pairs != 0;
   cudaLaunchAttribute attrs[2];
   std::memset(attrs, 0, sizeof(attrs));
   attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -808,7 +851,7 @@ cudaError_t launch_splitkv(const SplitKVParams& p, cudaStream_t stream) {
   attrs[1].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(p.num_parts, pair ? 2 : 1);
+  cfg.gridDim = dim3(p.num_parts, pair ? 2 : (p.h_q + kHeads - 1) / kHeads);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;

@@ -28,6 +28,7 @@ struct SplitKVParams {
   const int32_t* indices;       // [R][topk] (sparse mode)
   const int32_t* tile_prefix;   // [R + 1] tiles before each request (dense modes), or nullptr
   int kv_mode;                  // KvMode
+  int cta_pairs;                // 128 heads: 1 = two-CTA cluster sharing dequantised tiles, 0 = independent CTAs
   int causal;                   // dense modes: token t of s_q sees seqlen - (s_q - 1 - t) positions
   const int32_t* sched_meta;    // [num_parts][8]
   const int32_t* num_splits;    // [R + 1]
@@ -43,12 +44,12 @@ struct SplitKVParams {
 };
 
 // Heads merged by one CTA of the combine kernel (one warp per head).
-constexpr int kCombineHeadsPerCta = 8;
+constexpr int kCombineHeadsPerCta = 4;
 
 // Dynamic shared memory of the split kernel, its attribute set-up (for the
-// current device) and its launch (single CTA for <= 64 heads, a two-CTA
-// cluster for 128 heads; chained to the previous kernel with programmatic
-// dependent launch).
+// current device) and its launch (one CTA per part and 64-head group, or for
+// 128 heads with cta_pairs a two-CTA cluster per part; chained to the
+// previous kernel with programmatic dependent launch).
 int splitkv_smem_bytes();
 cudaError_t configure_splitkv();
 cudaError_t launch_splitkv(const SplitKVParams& p, cudaStream_t stream);
@@ -84,6 +85,9 @@ struct DecodeCall {
 // per host thread) and returns SMLA_ERR_CUDA.
 int cuda_failure(cudaError_t e);
 int g_last_cuda_error_value();
+
+// The process-wide form of 128-head decodes (smla_set_head_pair_form).
+int head_pair_form();
 
 // Scratch layout of a decode: a 256-byte status header, then float32
 // o_accum [max_splits][h_q][512] and lse_accum [max_splits][h_q], each

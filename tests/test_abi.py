@@ -36,9 +36,19 @@ def test_status_strings_and_version():
     assert L.smla_status_string(0) == b"SMLA_OK"
     assert L.smla_status_string(4) == b"SMLA_ERR_DEVICE_TIMEOUT"
     assert L.smla_status_string(99) == b"SMLA_UNKNOWN_STATUS"
-    assert L.smla_version() == 101
+    assert L.smla_version() == 102
     assert L.smla_last_cuda_error() == 0
     assert L.smla_last_cuda_error_string() == b"cudaSuccess"
+
+
+def test_head_pair_form_setting_round_trips():
+    # host-side only: the setting is read at the next decode launch
+    prev = smla.set_head_pair_form(True)
+    try:
+        assert smla.set_head_pair_form(False) is True
+        assert smla.set_head_pair_form(False) is False
+    finally:
+        smla.set_head_pair_form(prev)
 
 
 def test_workspace_bytes_arithmetic():
@@ -49,6 +59,7 @@ def test_workspace_bytes_arithmetic():
     l_bytes = (R + P) * h * 4
     rnd = lambda x: (x + 255) // 256 * 256
     assert L.smla_workspace_bytes(64, 1, 128, 2048, 74) == 256 + rnd(o_bytes) + rnd(l_bytes)
+    assert L.smla_workspace_bytes(3, 2, 16, 64, 5) == 256 + rnd(11 * 16 * 2048) + rnd(11 * 16 * 4)
     assert L.smla_workspace_bytes(2, 1, 48, 64, 8) == 0       # unsupported h_q
     assert L.smla_workspace_bytes(2, 0, 16, 64, 8) == 0       # s_q < 1
     assert L.smla_workspace_bytes(2, 1, 16, 0, 8) == 0        # topk < 1

@@ -145,6 +145,27 @@ def test_h128_long_topk_many_splits(smla):
     _check(w)
 
 
+@pytest.mark.parametrize("P", [None, 7], ids=["default_parts", "7_parts"])
+def test_h128_head_pair_form_matches_independent_ctas(smla, torch_cuda, P):
+    """The two-CTA cluster form (each CTA dequantises half of every tile and
+    copies it to its peer) and the default independent CTAs give bitwise
+    identical o and lse, and both pass the oracle comparison."""
+    import sparse_mla_decoding_b200 as m
+    w = W.Workload("h128_pairs", batch=3, s_q=2, h_q=128, topk=700, seed=93, seqlens=(3000, 900, 5000),
+                   index_mode="uniform", invalid_per_token=50)
+    hi = PU.build_host_inputs(w)
+    d = PU.to_device(hi)
+    o1, l1, _, _ = PU.run_gpu(hi, dev_inputs=d, num_sm_parts=P)
+    prev = m.set_head_pair_form(True)
+    try:
+        o2, l2, _, _ = PU.run_gpu(hi, dev_inputs=d, num_sm_parts=P)
+    finally:
+        m.set_head_pair_form(prev)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    toks = [(b, t) for b in range(w.batch) for t in range(w.s_q)]
+    PU.compare(o2, l2, PU.oracle_tokens(hi, toks), w.name + " pair form")
+
+
 def test_invalid_slots_and_all_invalid_tokens(smla):
     w = W.Workload("invalid", batch=3, s_q=2, h_q=64, topk=192, seed=5, seqlens=(300, 64, 1000),
                    index_mode="uniform")
