@@ -194,6 +194,19 @@ __device__ __forceinline__ void issue_pv_tile(uint32_t d_lo16, uint32_t d_hi16, 
       : "memory");
 }
 
+// (a.x * b + c, a.y * b + c) in one packed instruction, each a fused
+// multiply-add rounded exactly as fmaf.
+__device__ __forceinline__ float2 ffma2_rn(float2 a, float b, float c) {
+  uint64_t v, bb, cc, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(bb) : "f"(b));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(cc) : "f"(c));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(v), "l"(bb), "l"(cc));
+  float2 out;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(out.x), "=f"(out.y) : "l"(r));
+  return out;
+}
+
 // 2^x on the special-function unit (P is rounded to bf16 right after).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -467,21 +480,40 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
             const uint32_t qaddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + kQCol;
             const int c0 = (pw < 4) ? 0 : 5, c1 = (pw < 4) ? 5 : 9;
             // each chunk in two halves of 8 columns (the two 16-thread halves of
-            // the warp write 16 columns apart), to keep few registers live
+            // the warp write 16 columns apart); the loads of kQB halves are in
+            // flight together, few enough registers to stay live beside the
+            // pipeline's row data (BF16 rows hold twice the row data)
+            constexpr int kQB = kBf16 ? 1 : 2;
 #pragma unroll 1
-            for (int h = 2 * c0; h < 2 * c1; ++h) {
-              const int c = h >> 1, u0 = 2 * (h & 1);
-              uint32_t v[8];
+            for (int h = 2 * c0; h < 2 * c1; h += kQB) {
+              uint32_t v[kQB][8];
 #pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                uint4 x = make_uint4(0u, 0u, 0u, 0u);
-                ldg_v4_if(x, qrow + 64 * c + 32 * (lane >> 4) + 8 * (u0 + u), qlive);
-                v[4 * u] = x.x;
-                v[4 * u + 1] = x.y;
-                v[4 * u + 2] = x.z;
-                v[4 * u + 3] = x.w;
+              for (int g = 0; g < kQB; ++g) {
+                const int c = (h + g) >> 1, u0 = 2 * ((h + g) & 1);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                  uint4 x = make_uint4(0u, 0u, 0u, 0u);
+                  ldg_v4_if(x, qrow + 64 * c + 32 * (lane >> 4) + 8 * (u0 + u), qlive);
+                  v[g][4 * u] = x.x;
+                  v[g][4 * u + 1] = x.y;
+                  v[g][4 * u + 2] = x.z;
+                  v[g][4 * u + 3] = x.w;
+                }
               }
-              tmem_st16x2_8<16>(qaddr + 32 * c + 4 * u0, v);
+#pragma unroll
+              for (int g = 0; g < kQB; ++g) {
+                const int c = (h + g) >> 1, u0 = 2 * ((h + g) & 1);
+                tmem_st16x2_8<16>(qaddr + 32 * c + 4 * u0, v[g]);
+              }
+            }
+            // The next request's rows of Q into L2 now, so its staging (on the
+            // pipeline's critical path: S waits for it) reads L2, not DRAM.
+            // (Not with BF16 rows: their row data leaves no registers for it.)
+            if (!kBf16 && cf.r + 1 < p.num_requests) {
+              const char* qn = reinterpret_cast<const char*>(p.q + ((size_t)(cf.r + 1) * p.h_q + (size_t)kHeads * hg) * 576);
+              const int nlines = heads_here * 576 * 2 / 128;
+#pragma unroll 1
+              for (int i = 32 * pw + lane; i < nlines; i += 32 * kProducerWarps) prefetch_l2_if(qn + 128 * i, true);
             }
           }
           tmem_wait_st();
@@ -704,10 +736,22 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       uint32_t sr[32];
       tmem_ld16x2_32(tmem + t_lane + kSCol + 64 * s, sr);
       tmem_wait_ld();
+      // Tiles whose 64 slots are all valid (the usual case) skip the
+      // per-column mask tests; the results are the same either way.
+      const bool all_valid = __all_sync(0xffffffffu, vh == 0xFFFFFFFFu);
       float mt = -INFINITY;
+      if (all_valid) {
+        float mx[8];
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
-        if ((vh >> c) & 1u) mt = fmaxf(mt, __uint_as_float(sr[c]));
+        for (int c = 0; c < 8; ++c)
+          mx[c] = fmaxf(fmaxf(__uint_as_float(sr[4 * c]), __uint_as_float(sr[4 * c + 1])),
+                        fmaxf(__uint_as_float(sr[4 * c + 2]), __uint_as_float(sr[4 * c + 3])));
+        mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if ((vh >> c) & 1u) mt = fmaxf(mt, __uint_as_float(sr[c]));
+      }
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
       float alpha = 1.f;
       mt = (mt == -INFINITY) ? -INFINITY : mt * scale_log2;
@@ -720,13 +764,25 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
       float psum = 0.f;
       uint32_t pk[16];
+      if (all_valid) {
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float p0 = ((vh >> (2 * c)) & 1u) ? fast_exp2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, neg_m)) : 0.f;
-        const float p1 =
-            ((vh >> (2 * c + 1)) & 1u) ? fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, neg_m)) : 0.f;
-        psum += p0 + p1;
-        pk[c] = bf162_bits(__floats2bfloat162_rn(p0, p1));
+        for (int c = 0; c < 16; ++c) {
+          const float2 t = ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale_log2,
+                                    neg_m);
+          const float p0 = fast_exp2(t.x), p1 = fast_exp2(t.y);
+          psum += p0 + p1;
+          pk[c] = bf162_bits(__floats2bfloat162_rn(p0, p1));
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float p0 =
+              ((vh >> (2 * c)) & 1u) ? fast_exp2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, neg_m)) : 0.f;
+          const float p1 =
+              ((vh >> (2 * c + 1)) & 1u) ? fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, neg_m)) : 0.f;
+          psum += p0 + p1;
+          pk[c] = bf162_bits(__floats2bfloat162_rn(p0, p1));
+        }
       }
       if (m_used != -INFINITY) l_half += psum;
       // An O rescale needs PV(j - 1) complete (this warpgroup issues every PV,
