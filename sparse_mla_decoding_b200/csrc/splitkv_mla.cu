@@ -728,8 +728,10 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         req_ok = !(ns_r < 0 || ns_r1 > p.max_splits || nsplit < 1 || slot < ns_r || slot >= ns_r1);
         if (!req_ok && tid == 0) report_status(p.status, kStatusBadSchedule);
       }
-      if (!mbar_wait_bounded_warp(&tail->sfull[s], ph, kWaitLimitNs, p.status)) break;
+      // The tile's validity bytes are published with kfull, which completes
+      // before S(j) is even issued: wait for it first, while S executes.
       if (!mbar_wait_bounded_warp(&tail->kfull[s], ph, kWaitLimitNs, p.status)) break;
+      if (!mbar_wait_bounded_warp(&tail->sfull[s], ph, kWaitLimitNs, p.status)) break;
       tc_fence_after();
       // validity bits of this thread's 32 columns (one nibble per 4 rows)
       const uint32_t vh = nibbles_to_bits(ld_shared_u64(smem_u32(&tail->vmask[s][8 * half])));
