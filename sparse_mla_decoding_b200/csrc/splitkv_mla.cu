@@ -115,8 +115,8 @@ struct __align__(16) Tail {
   uint64_t kfull[2];   // K tile s written (producers of both CTAs of a pair)
   uint64_t kempty[2];  // K tile s consumed by PV (both CTAs of a pair)
   uint64_t sfull[2];   // S buffer s computed
-  uint64_t ofree;      // PV complete
-  uint64_t pready;     // the four softmax warps stored P (phase j for tile j)
+  uint64_t ofree[2];   // PV(j) complete, for tile j in ring slot j % 2
+  uint64_t pready[2];  // the four softmax warps stored P(j), for tile j in ring slot j % 2
   uint64_t qfull;      // Q tile loaded
   uint64_t qfree;      // last S of a request complete: sQ reusable
   uint32_t tmem_base;
@@ -358,8 +358,10 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       mbar_init(&tail->kempty[s], kPair ? 2 : 1);
       mbar_init(&tail->sfull[s], 1);
     }
-    mbar_init(&tail->ofree, 1);
-    mbar_init(&tail->pready, 4);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&tail->ofree[s], 1);
+      mbar_init(&tail->pready[s], 4);
+    }
     mbar_init(&tail->qfull, 32 * kProducerWarps);
     mbar_init(&tail->qfree, 1);
     fence_mbarrier_init();
@@ -787,10 +789,15 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
         }
       }
       if (m_used != -INFINITY) l_half += psum;
-      // An O rescale needs PV(j - 1) complete (this warpgroup issues every PV,
-      // so the parity of ofree's current phase cannot run ahead of j - 1).
+      // An O rescale needs PV(j - 1) complete.  The PV barriers are per ring
+      // slot, which makes every such wait unambiguous: a warp that sees S(j)
+      // knows PV(j - 2) completed (its ring slot was refilled for tile j), so
+      // ofree[slot of j - 1] is at most one phase short of PV(j - 1).  (With
+      // one barrier for all tiles a warp running ahead could match the parity
+      // of a phase two PVs old.)
       if (!tp.first && __any_sync(0xffffffffu, alpha != 1.f)) {
-        if (!mbar_wait_bounded_warp(&tail->ofree, (uint32_t)((j - 1) & 1), kWaitLimitNs, p.status)) break;
+        if (!mbar_wait_bounded_warp(&tail->ofree[s ^ 1], (uint32_t)(((j - 1) >> 1) & 1), kWaitLimitNs, p.status))
+          break;
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
@@ -810,19 +817,19 @@ __global__ void __launch_bounds__(kRegCapThreads, 1) splitkv_mla_kernel(const Sp
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tail->pready);
+      if (lane == 0) mbar_arrive(&tail->pready[s]);
       if (warp == 0) {
-        if (!mbar_spin_bounded_warp(&tail->pready, (uint32_t)(j & 1), kWaitLimitNs, p.status)) break;
+        if (!mbar_spin_bounded_warp(&tail->pready[s], (uint32_t)((j >> 1) & 1), kWaitLimitNs, p.status)) break;
         tc_fence_after();
         issue_pv_tile(tmem + (kOLane << 16), tmem + (kOLane << 16) + 256, p_lo0 + (uint32_t)s * (kAtom >> 4),
                       v_lo0 + (uint32_t)s * (kTileBytes >> 4), d_hi, idesc_pv, tp.first ? 0u : 1u);
         if (kPair) mma_commit_multicast(&tail->kempty[s], (uint16_t)0x3);
         else mma_commit(&tail->kempty[s]);
-        mma_commit(&tail->ofree);
+        mma_commit(&tail->ofree[s]);
       }
 
       if (tp.last) {
-        if (!mbar_wait_bounded_warp(&tail->ofree, (uint32_t)(j & 1), kWaitLimitNs, p.status)) break;
+        if (!mbar_wait_bounded_warp(&tail->ofree[s], (uint32_t)((j >> 1) & 1), kWaitLimitNs, p.status)) break;
         tc_fence_after();
         const float l_me = l_half + __shfl_xor_sync(0xffffffffu, l_half, 16);
         const float m_me = m_used;
