@@ -229,6 +229,25 @@ def test_bitwise_deterministic(smla, torch_cuda):
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
+def test_repeated_calls_with_many_request_ends_are_bitwise_identical(smla, torch_cuda):
+    """Requests of one or two tiles put an epilogue (a wait for the last PV, then
+    O read out of TMEM) on almost every tile, with split requests on both sides of
+    every part boundary: the pattern where a softmax warp running ahead of the PV
+    issuer could read O early.  Repeated calls must agree bit for bit, and the
+    first must pass the oracle comparison."""
+    w = W.Workload("many_ends", batch=96, s_q=1, h_q=128, topk=96, seed=14, seqlens=tuple([300, 70, 1500] * 32),
+                   index_mode="uniform", invalid_per_token=9)
+    hi = PU.build_host_inputs(w)
+    d = PU.to_device(hi)
+    o1, l1, _, ns = PU.run_gpu(hi, dev_inputs=d, num_sm_parts=39)   # 5 tiles a part: every other boundary splits
+    assert (np.diff(ns) > 1).any(), "expected split requests"
+    for _ in range(4):
+        o2, l2, _, _ = PU.run_gpu(hi, dev_inputs=d, num_sm_parts=39)
+        assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    toks = [(b, 0) for b in range(0, w.batch, 7)]
+    PU.compare(o1, l1, PU.oracle_tokens(hi, toks), w.name)
+
+
 def test_dequant_every_code_and_scale_range_is_exact(smla, torch_cuda):
     """A single valid slot makes o equal its value row exactly, so o exposes the
     dequantised latent values: every e4m3 code (NaN codes included) times
