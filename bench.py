@@ -680,6 +680,29 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     kern_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
 
+    # ---- the same decode calls in the two-CTA cluster form (128 heads), for comparison
+    cluster_form = None
+    if w.h_q > 64:
+        prev_form = smla.set_head_pair_form(True)
+        try:
+            torch.cuda.synchronize()
+            for i in range(args.steps):
+                d, (sm, ns) = copies[i % args.copies], metas[i % args.copies]
+                evs[i][0].record(stream)
+                smla.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"],
+                                            sm, ns, workspace=ws, out=outs)
+                evs[i][1].record(stream)
+            torch.cuda.synchronize()
+            pair_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+            cluster_form = {"kernel_ms": pair_ms,
+                            "decode_call_tflops": float(np.mean(flops_per_copy)) / (pair_ms * 1e-3) / 1e12,
+                            "note": "smla_set_head_pair_form(1): each 128-head part as a two-CTA cluster sharing "
+                                    "dequantised tiles; the default runs the two 64-head CTAs independently"}
+        except Exception as e:   # a comparison only: never lose the bench line over it
+            cluster_form = {"error": f"{type(e).__name__}: {e}"}
+        finally:
+            smla.set_head_pair_form(prev_form)
+
     # ---- end to end: pinned host inputs in, results out, every step --------
     e2e = None
     host = []
@@ -767,6 +790,8 @@ def run_ours(args, w, rank, world, local_rank):
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,
     }
+    if cluster_form is not None:
+        line["cluster_form"] = cluster_form
     if world == 1 and not args.no_cpu_baseline:
         hi = host_inputs(w.with_(seed=w.seed))
         f, t, n = cpu_oracle_sample(w, hi, args.cpu_seconds)
