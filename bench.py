@@ -253,6 +253,23 @@ def run_reference(args, w, rank, world):
 # our arm
 # ---------------------------------------------------------------------------
 
+def time_decode_calls(smla, torch, copies, metas, ws, outs, stream, steps):
+    """Mean CUDA-event duration (ms) of `steps` decode calls over the rotating input copies.
+
+    Each call is bracketed by its own pair of events on `stream`; the device is
+    synchronised before and after the loop."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        d, (sm, ns) = copies[i % len(copies)], metas[i % len(metas)]
+        evs[i][0].record(stream)
+        smla.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"], sm, ns,
+                                    workspace=ws, out=outs)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+
 def make_device_copy(w, device, values="host"):
     """Generator values -> device tensors; the cache rows are written by the library's own KV writer.
 
@@ -667,37 +684,17 @@ def run_ours(args, w, rank, world, local_rank):
     my_valid = sum(valid_per_copy[i % args.copies] for i in range(args.steps))
 
     # ---- the decode call alone (split kernel + chained combine), for the roofline
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     metas = [smla.get_mla_metadata(copies[c]["cache_seqlens"], topk, w.h_q, num_parts, s_q=w.s_q)
              for c in range(args.copies)]
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        d, (sm, ns) = copies[i % args.copies], metas[i % args.copies]
-        evs[i][0].record(stream)
-        smla.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"], sm, ns,
-                                    workspace=ws, out=outs)
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    kern_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    kern_ms = time_decode_calls(smla, torch, copies, metas, ws, outs, stream, args.steps)
 
     # ---- the same decode calls in the two-CTA cluster form (128 heads), for comparison
     cluster_form = None
     if w.h_q > 64:
         prev_form = smla.set_head_pair_form(True)
         try:
-            for i in range(3):   # warm-up of this form
-                d, (sm, ns) = copies[i % args.copies], metas[i % args.copies]
-                smla.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"],
-                                            sm, ns, workspace=ws, out=outs)
-            torch.cuda.synchronize()
-            for i in range(args.steps):
-                d, (sm, ns) = copies[i % args.copies], metas[i % args.copies]
-                evs[i][0].record(stream)
-                smla.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], d["indices"],
-                                            sm, ns, workspace=ws, out=outs)
-                evs[i][1].record(stream)
-            torch.cuda.synchronize()
-            pair_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+            time_decode_calls(smla, torch, copies, metas, ws, outs, stream, 3)   # warm-up of this form
+            pair_ms = time_decode_calls(smla, torch, copies, metas, ws, outs, stream, args.steps)
             cluster_form = {"kernel_ms": pair_ms,
                             "decode_call_tflops": float(np.mean(flops_per_copy)) / (pair_ms * 1e-3) / 1e12,
                             "note": "smla_set_head_pair_form(1): each 128-head part as a two-CTA cluster sharing "

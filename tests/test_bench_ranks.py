@@ -126,3 +126,46 @@ def test_clock_sampler_without_timestamps_uses_every_sample():
     c.mark_end()
     s = c.summarize(rows)
     assert s["samples"] == 1 and s["sm_mhz"] == 1800.0 and "whole sampler run" in s["window"]
+
+
+def test_time_decode_calls_brackets_each_call_and_rotates_copies():
+    """The roofline's decode-call timing (also used for the cluster-form comparison):
+    one event pair per call on the given stream, copies and metadata rotated, the
+    device synchronised around the loop, the mean of the per-call durations."""
+    import bench
+
+    log = []
+
+    class Event:
+        t = 0.0
+
+        def __init__(self, enable_timing):
+            assert enable_timing
+            self.when = None
+
+        def record(self, stream):
+            assert stream == "s0"
+            Event.t += 1.0
+            self.when = Event.t
+            log.append("rec")
+
+        def elapsed_time(self, other):
+            return other.when - self.when
+
+    fake_torch = types.SimpleNamespace(cuda=types.SimpleNamespace(
+        Event=Event, synchronize=lambda: log.append("sync")))
+
+    class FakeLib:
+        def flash_mla_with_kvcache(self, q, kv, bt, sl, idx, sm, ns, workspace, out):
+            assert workspace == "ws" and out == "outs"
+            log.append(("call", q, sm))
+            Event.t += 2.0      # each call takes 2 units between its two records
+
+    copies = [dict(q=f"q{c}", kvcache="kv", block_table="bt", cache_seqlens="sl", indices="idx") for c in range(3)]
+    metas = [(f"sm{c}", "ns") for c in range(3)]
+    ms = bench.time_decode_calls(FakeLib(), fake_torch, copies, metas, "ws", "outs", "s0", 5)
+    assert ms == 3.0            # record, +2 for the call, record: 3 units per call
+    calls = [e for e in log if isinstance(e, tuple)]
+    assert [c[1] for c in calls] == ["q0", "q1", "q2", "q0", "q1"]
+    assert [c[2] for c in calls] == ["sm0", "sm1", "sm2", "sm0", "sm1"]
+    assert log[0] == "sync" and log[-1] == "sync" and log.count("rec") == 10
