@@ -78,6 +78,23 @@ def test_dense_decode_parity(w, causal, kv_format):
     PU.compare(o, lse, ref, f"{w.name} {'causal' if causal else 'full'} {'bf16' if kv_format else 'fp8'}")
 
 
+@pytest.mark.parametrize("kv_format", [oracle.KV_FP8, oracle.KV_BF16], ids=["fp8", "bf16"])
+def test_dense_h128_cluster_form_matches_default(kv_format):
+    """The two-CTA cluster form of 128-head decodes (smla.set_head_pair_form) in
+    the dense modes: bitwise equal to the default independent CTAs."""
+    import sparse_mla_decoding_b200 as smla
+    w = SHAPES[2]                    # dense_h128_varlen
+    hi = build(w, kv_format)
+    o1, l1, *_ , (st1, _) = run(hi, w, kv_format, True)
+    prev = smla.set_head_pair_form(True)
+    try:
+        o2, l2, *_, (st2, _) = run(hi, w, kv_format, True)
+    finally:
+        smla.set_head_pair_form(prev)
+    assert st1 == 0 and st2 == 0
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
 @pytest.mark.parametrize("parts", [1, 3, 148])
 def test_dense_split_schedules(parts):
     """Every split count gives the same answer within the tolerances (one part: no combine)."""
